@@ -1,0 +1,371 @@
+"""Throughput of the H3-Omni block step on B200: packed tokens/s per block.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = the whole hot path once over one packed sequence: patchify + pack +
+per-modality input projections, one full-width block (LN+modulate, QKV with
+Q/K RMSNorm + 3-D RoPE, attention, gated out-projection, LN+modulate, gated
+SwiGLU FFN), the output head and the two Euler updates (video, audio).
+Every rank processes its own sequence (independent requests, no collective):
+weak scaling, value = tokens of all ranks / max-over-ranks time.
+
+--impl reference times the float64 CPU oracle on a bounded sample of the same
+workload (the reference arm of this comparison; it is not tuned).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed tokens/s per Omni block (bf16, 1×B200) & % of dense bf16 tensor peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "768sq_2s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def flops_per_call(w, L):
+    """Algorithmic FLOPs of each C-ABI call at L valid tokens (no padding)."""
+    D, I, F = w.D, w.I, w.F
+    return {
+        "h3_qkv_qknorm_mrope": 2.0 * L * D * 3 * I,
+        "h3_attention": 4.0 * L * L * I,
+        "h3_gated_residual": 2.0 * L * I * D,
+        "h3_ffn_swiglu": 2.0 * L * D * 2 * F + 2.0 * L * F * D,
+    }
+
+
+def bytes_per_call(w, L, Lp):
+    """Algorithmic HBM bytes of the memory-bound calls."""
+    D = w.D
+    n_lat = w.T_lat * w.H_lat * w.W_lat * w.C_lat + w.audio_channels * w.n_audio * w.C_audio
+    return {
+        "h3_adaln_norm_modulate": L * (4 * D + 2 * D) + (Lp - L) * 2 * D,
+        "h3_euler_step": 12 * n_lat,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) == 7:
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                except ValueError:
+                    pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    from omni_modal_diffusion_b200 import h3
+    from omni_modal_diffusion_b200.pipeline import H3BlockStep
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + w.index + 7919 * rank)
+
+    def randn(*shape, std=1.0, dtype=torch.bfloat16):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(dtype)
+
+    # random-init weights of the block's architecture, N(0, 0.02), bf16
+    W = {"W_text": randn(w.D, w.D_text, std=0.02), "W_vid": randn(w.D, 4 * w.C_lat, std=0.02),
+         "W_aud": randn(w.D, w.C_audio, std=0.02), "Wqkv": randn(3 * w.I, w.D, std=0.02),
+         "qn_w": (1 + 0.1 * torch.randn(128, generator=g, device=dev)).to(torch.bfloat16),
+         "kn_w": (1 + 0.1 * torch.randn(128, generator=g, device=dev)).to(torch.bfloat16),
+         "Wo": randn(w.D, w.I, std=0.02), "Wgu": randn(2 * w.F, w.D, std=0.02), "Wd": randn(w.D, w.F, std=0.02),
+         "W_vhead": randn(4 * w.C_lat, w.D, std=0.02), "W_ahead": randn(w.C_audio, w.D, std=0.02)}
+    st = H3BlockStep(w, device=dev, weights=W)
+    L, Lp = st.ranges.L, st.ranges.L_pad
+    text = randn(w.n_text, w.D_text)
+    video = randn(w.T_lat, w.H_lat, w.W_lat, w.C_lat)
+    audio = randn(w.audio_channels, w.n_audio, w.C_audio)
+    mod = randn(3, 6, w.D, std=0.1, dtype=torch.float32)
+    lat_v = randn(w.T_lat, w.H_lat, w.W_lat, w.C_lat, dtype=torch.float32)
+    lat_a = randn(w.audio_channels, w.n_audio, w.C_audio, dtype=torch.float32)
+    sv = h3.h3_sigma_schedule(8, 12.0)
+    sa = h3.h3_sigma_schedule(8, 3.0)
+    stream = torch.cuda.current_stream(dev)
+
+    calls = ["h3_embed_pack", "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
+             "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step"]
+
+    def step(i, ev=None):
+        s = i % 8
+        mark = (lambda k, j: ev[k][j].record(stream)) if ev is not None else (lambda k, j: None)
+        d, r = st.dims, st.ranges
+        mark(0, 0); st.embed(text, video, audio); mark(0, 1)
+        mark(1, 0); h3.h3_adaln_norm_modulate(d, r, st.x, mod, h3.H3_MSA, st.xm); mark(1, 1)
+        mark(2, 0)
+        h3.h3_qkv_qknorm_mrope(d, r, st.xm, st.W["Wqkv"], st.W["qn_w"], st.W["kn_w"], st.pos, st.q, st.k, st.v)
+        mark(2, 1)
+        mark(3, 0); h3.h3_attention(d, r, st.q, st.k, st.v, st.o); mark(3, 1)
+        mark(4, 0); h3.h3_gated_residual(d, r, st.x, st.o, st.W["Wo"], mod, h3.H3_MSA); mark(4, 1)
+        mark(5, 0); h3.h3_adaln_norm_modulate(d, r, st.x, mod, h3.H3_MLP, st.xm); mark(5, 1)
+        mark(6, 0); h3.h3_ffn_swiglu(d, r, st.x, st.xm, st.W["Wgu"], st.W["Wd"], mod, st.ws); mark(6, 1)
+        mark(7, 0); st.head(); mark(7, 1)
+        mark(8, 0); st.euler(lat_v, lat_a, (sv[s], sv[s + 1]), (sa[s], sa[s + 1])); mark(8, 1)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    sampler = ClockSampler(local) if rank == 0 or world == 1 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in calls] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i, ev[i])
+    t1.record(stream)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_total = t0.elapsed_time(t1)
+    per_call = {c: statistics.mean(ev[i][k][0].elapsed_time(ev[i][k][1]) for i in range(args.steps))
+                for k, c in enumerate(calls)}
+    status = h3.h3_device_status()
+    if status != 0:
+        raise RuntimeError(f"device-side wait gave up (code {status})")
+
+    # ---- end to end: host buffers in pinned memory, H2D + step + D2H in the timed region
+    host_in = {k: t.cpu().pin_memory() for k, t in (("text", text), ("video", video), ("audio", audio), ("mod", mod),
+                                                      ("lat_v", lat_v), ("lat_a", lat_a))}
+    dev_in = {k: torch.empty_like(t, device=dev) for k, t in host_in.items()}
+    host_out = {k: torch.empty_like(host_in[k]).pin_memory() for k in ("lat_v", "lat_a")}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def e2e_step(i):
+        for k in host_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        s = i % 8
+        st.step(dev_in["text"], dev_in["video"], dev_in["audio"], dev_in["mod"], dev_in["lat_v"], dev_in["lat_a"],
+                (sv[s], sv[s + 1]), (sa[s], sa[s + 1]))
+        host_out["lat_v"].copy_(dev_in["lat_v"], non_blocking=True)
+        host_out["lat_a"].copy_(dev_in["lat_a"], non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+
+    # max over ranks
+    vals = torch.tensor([ms_total, ms_e2e], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, ms_e2e = vals.tolist()
+    per_call_t = torch.tensor([per_call[c] for c in calls], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(per_call_t, op=dist.ReduceOp.MAX)
+        dist.destroy_process_group()
+    per_call = dict(zip(calls, per_call_t.tolist()))
+    if rank != 0:
+        return None
+
+    ms_step = ms_total / args.steps
+    value = world * L / (ms_step / 1e3)
+    e2e_value = world * L / (ms_e2e / args.steps / 1e3)
+    peaks = _peaks()
+    fl = flops_per_call(w, L)
+    by = bytes_per_call(w, L, Lp)
+    tensor_calls = {c: fl[c] / (per_call[c] / 1e3) / 1e12 for c in fl}
+    dominant = max(fl, key=lambda c: per_call[c])
+    peak_tf = peaks["bf16_tflops_sustained"]
+    block_flops = sum(fl.values())
+    block_ms = sum(per_call[c] for c in ("h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
+                                         "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu"))
+    ln_gbs = by["h3_adaln_norm_modulate"] / (per_call["h3_adaln_norm_modulate"] / 1e3) / 1e9
+    launches = st.launches_per_step()
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/text, N(0,0.02) random-init weights)",
+        "config": {"workload": w.name, "packed_tokens": L, "L_pad": Lp, "hidden": w.D, "heads": w.H, "head_dim": 128,
+                   "ffn": w.F, "text_tokens": w.n_text, "audio_tokens": w.audio_channels * w.n_audio,
+                   "video_tokens": st.n_video, "video_latent": [w.T_lat, w.H_lat, w.W_lat, w.C_lat],
+                   "parallelism": f"replicas x{world} (independent sequences)",
+                   "l2": "inputs larger than L2: %.0f MB of weights + %.0f MB residual stream read per step" % (
+                       sum(t.numel() * 2 for t in W.values()) / 1e6, Lp * w.D * 4 / 1e6)},
+        "roofline": {"bound": "tensor", "kernel": dominant,
+                     "achieved": round(tensor_calls[dominant], 1),
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(tensor_calls[dominant] / peak_tf, 4),
+                     "peak_kind": f"bf16 sustained ({peaks['source']})",
+                     "traffic": None},
+        "block": {"tflops": round(block_flops / (block_ms / 1e3) / 1e12, 1),
+                  "frac_of_bf16_sustained": round(block_flops / (block_ms / 1e3) / 1e12 / peak_tf, 4),
+                  "frac_of_bf16_spec_2250": round(block_flops / (block_ms / 1e3) / 1e12 / 2250.0, 4),
+                  "ms": round(block_ms, 4)},
+        "per_call_ms": {c: round(v, 4) for c, v in per_call.items()},
+        "per_call_tflops": {c: round(v, 1) for c, v in tensor_calls.items()},
+        "ln_modulate_gbs": round(ln_gbs, 1), "ln_modulate_frac_hbm": round(ln_gbs / peaks["hbm_gbs"], 4),
+        "gpu_launches": launches * args.steps,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
+    return out
+
+
+def cpu_baseline(w, rows_sample=32):
+    """The float64 oracle on the host cores, on a bounded sample of the same
+    workload: K and V of every token (all of them feed attention) plus the
+    full block for `rows_sample` query rows; the per-row part is scaled to all
+    L rows (the block's cost is exactly K/V for all tokens + per-row work)."""
+    from oracle import h3_oracle as O
+    from omni_modal_diffusion_b200 import synthetic as S
+    try:
+        import threadpoolctl
+        threads = max(info.get("num_threads", 0) for info in threadpoolctl.threadpool_info()) or os.cpu_count()
+    except Exception:  # pragma: no cover
+        threads = os.cpu_count()
+    inp = S.make_inputs(w)
+    t_g, i_g, j_g = O.token_grid(w.T_lat, w.H_lat, w.W_lat)
+    r = O.pack_ranges(w.n_text, w.audio_channels * w.n_audio, t_g * i_g * j_g)
+    pos = O.positions(r, t_g, i_g, j_g, w.audio_channels, w.n_audio)
+    x = O.embed(inp["text"], inp["video"], inp["audio"], inp["W_text"], inp["W_vid"], inp["W_aud"], r)
+    L = r["L"]
+    rows = S.random_rows(L, rows_sample, seed=99)
+    t0 = time.perf_counter()
+    O.block_forward_rows(x, inp["mod"], r, pos, rows[:1], inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"],
+                         inp["Wgu"], inp["Wd"], w.H)
+    t_kv = time.perf_counter() - t0       # K/V for all tokens + 1 row
+    t0 = time.perf_counter()
+    O.block_forward_rows(x, inp["mod"], r, pos, rows, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"],
+                         inp["Wgu"], inp["Wd"], w.H)
+    t_all = time.perf_counter() - t0
+    per_row = max(t_all - t_kv, 1e-9) / (len(rows) - 1)
+    t_block = (t_kv - per_row) + per_row * L
+    return {"value": round(L / t_block, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"float64 oracle block on {w.name}: K/V of all {L} tokens + {len(rows)} sampled query rows "
+                      f"({t_kv + t_all:.1f} s measured), per-row time scaled to {L} rows",
+            "seconds_per_block_extrapolated": round(t_block, 2)}
+
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    vals, secs = [], []
+    base = None
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        cb = cpu_baseline(w, args.cpu_rows)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            vals.append(cb["value"])
+            secs.append(dt)
+            base = cb
+    value = statistics.mean(vals)
+    return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": {"workload": w.name},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": base["cores"], "kind": "oracle",
+                             "sample": base["sample"]},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=24)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference" and args.warmup > 1:
+        args.warmup = 1            # each oracle step is a ~10-30 s CPU sample
+    from omni_modal_diffusion_b200 import synthetic as S
+    w = S.WORKLOADS[args.workload]
+    out = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+/*
+ * h3.h -- C ABI of the B200 (sm_100a) H3-Omni block step.
+ *
+ * One forward pass of the single-stream H3-Omni-Transformer block over a
+ * packed text + audio + video token sequence, plus the flow-sampler Euler
+ * step.  Sources (page title, section):
+ *   [shouss] "MiniMax-H3: native joint audio-video generation"
+ *            (note.shouss.top): §2.2 packed sequence, §3 trunk with modality
+ *            modulation, §3.1 three modulation groups (6D per modality, 18D
+ *            total), §3.2 config table, Q/K RMSNorm then RoPE, SiLU(gate)*up,
+ *            §4.1 patch width, §4.3 AudioVAE, §5 non-causal attention and
+ *            update mask, §6 velocity sampling with video/audio schedulers.
+ *   [gojay]  "MiniMax-H3 paper reading" (gojay.top): §4 f16t4d24 VAE and
+ *            1x2x2 patchify, §5 Omni-Transformer, §7.3 shapes, §7.4 3-D
+ *            MM-RoPE (audio on the time axis only).
+ *   [0539]   "H3's omni-modal ambition" (0539edu.com): scheduler sigma
+ *            shifts 12.0 (video) and 3.0 (audio).
+ *
+ * Conventions (all entry points):
+ *   - Tensor arguments are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or synchronises device memory; every call is
+ *     asynchronous on the caller's stream (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).
+ *   - bf16 tensors are passed as h3_bf16 (the 16-bit pattern).  Weights are
+ *     row-major [out, in]; activations are row-major, one token per row.
+ *   - Every call validates all arguments before launching anything and
+ *     returns H3_OK or a negative status; on error nothing is launched and
+ *     h3_last_error() (per host thread) describes the problem.
+ *   - Pointers must be 16-byte aligned.  L_pad must be a multiple of 128.
+ *   - Modality ids / range order: text = 0, audio = 1, video = 2 (the packing
+ *     order text -> audio -> target video -> padding of [shouss] §2.2).
+ *   - Residual stream x: fp32 [L_pad][D]; rows >= L are padding (zero).
+ *   - Modulation mod: fp32 [3][6][D], per modality (shift_msa, scale_msa,
+ *     gate_msa, shift_mlp, scale_mlp, gate_mlp) ([shouss] §3.1).
+ */
+#ifndef H3_H
+#define H3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t h3_bf16;
+
+enum h3_status {
+  H3_OK = 0,
+  H3_ERR_NULL = -1,        /* a required pointer is NULL */
+  H3_ERR_SHAPE = -2,       /* inconsistent sizes or ranges */
+  H3_ERR_ALIGN = -3,       /* pointer not 16-byte aligned */
+  H3_ERR_UNSUPPORTED = -4, /* head_dim != 128, D % 64 != 0, F % 128 != 0, ... */
+  H3_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
+  H3_ERR_TIMEOUT = -6      /* a device-side wait gave up (see h3_device_status) */
+};
+
+enum h3_modality { H3_TEXT = 0, H3_AUDIO = 1, H3_VIDEO = 2 };
+enum h3_branch { H3_MSA = 0, H3_MLP = 1 };
+
+/* h3_qkv_qknorm_mrope / h3_attention flag: Q/K RMSNorm and RoPE are applied
+ * in the QKV GEMM epilogue (once per token), and h3_attention consumes the
+ * already-rotated q, k.  Required in this version. */
+#define H3_QK_NORM_ROPE_IN_QKV 1
+
+/* Block dimensions.  head_dim must be 128; I = H * head_dim;
+ * rope_t + rope_h + rope_w = head_dim, each even ([gojay] §7.4).
+ * theta: RoPE base (10000); eps_ln: LayerNorm epsilon; eps_qk: Q/K RMSNorm
+ * epsilon. */
+typedef struct h3_dims {
+  int D, H, head_dim, I, F;
+  int rope_t, rope_h, rope_w;
+  float theta, eps_ln, eps_qk;
+} h3_dims;
+
+/* Packed-sequence ranges: rows [start[m], start[m] + count[m]) hold modality
+ * m; the three ranges tile [0, L) without overlap; L_pad = L rounded up to a
+ * multiple of 128 ([shouss] §2.2). */
+typedef struct h3_ranges {
+  int start[3];
+  int count[3];
+  int L;
+  int L_pad;
+} h3_ranges;
+
+/* Description of the last error on this host thread (never NULL). */
+const char* h3_last_error(void);
+
+/* ABI version (major * 100 + minor). */
+int h3_version(void);
+
+/* Host only.  Fill `out` for n_text text tokens, n_audio_tokens audio tokens
+ * (channels x latents, channel-major) and n_video_tokens video tokens packed
+ * text -> audio -> video, L_pad = ceil(L / 128) * 128 ([shouss] §2.2). */
+int h3_make_ranges(int n_text, int n_audio_tokens, int n_video_tokens, h3_ranges* out);
+
+/* Host only.  n_steps + 1 sigmas from 1 to 0, uniform then time-shifted,
+ * sigma' = shift * sigma / (1 + (shift - 1) * sigma) (video shift 12.0,
+ * audio shift 3.0: [shouss] §6, [0539]).  out: host float[n_steps + 1]. */
+int h3_sigma_schedule(int n_steps, float shift, float* out);
+
+/* A1 + A2.  Patchify the video latent (1x2x2 over (t, h, w): token (t, i, j)
+ * takes latent pixels (t, 2i+ph, 2j+pw), feature (ph*2 + pw)*C_lat + c,
+ * [gojay] §4, §7.3), write token positions and modality ids, and project
+ * every modality into the residual stream with its own input projection
+ * ([gojay] §5: modality-specific parameters only in the I/O layers).
+ *   text     [count[TEXT]][D_text]               bf16
+ *   video    [T][Hl][Wl][C_lat] channels-last     bf16 (Hl, Wl even; C_lat % 4 == 0)
+ *   audio    [audio_channels][n_audio][C_audio]   bf16 (token = ch * n_audio + k)
+ *   W_text [D][D_text], W_vid [D][4*C_lat], W_aud [D][C_audio]  bf16
+ *   patches  workspace [count[VIDEO]][4*C_lat]     bf16 (caller-owned scratch;
+ *            holds the patch rows afterwards)
+ *   x_out    [L_pad][D] fp32 (rows >= L zeroed)
+ *   pos_out  [L_pad][3] fp32: video (t, i, j); audio latent k at (6k/40, 0, 0),
+ *            the 24/4 Hz video-latent time axis shared with 40 Hz audio
+ *            ([gojay] §7.4); text and padding (0, 0, 0)
+ *   mod_out  [L_pad] uint8 modality id, 255 for padding
+ * Requires count[VIDEO] == T * (Hl/2) * (Wl/2) and
+ * count[AUDIO] == audio_channels * n_audio. */
+int h3_embed_pack(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* text, int D_text,
+                  const h3_bf16* video, int T, int Hl, int Wl, int C_lat, const h3_bf16* audio,
+                  int audio_channels, int n_audio, int C_audio, const h3_bf16* W_text, const h3_bf16* W_vid,
+                  const h3_bf16* W_aud, h3_bf16* patches, float* x_out, float* pos_out, uint8_t* mod_out,
+                  void* stream);
+
+/* A3 / A8.  xm = LayerNorm(x) * (1 + scale_m) + shift_m, m = modality of the
+ * row's range, branch H3_MSA or H3_MLP selects the (shift, scale) pair
+ * ([shouss] §3, §3.1).  LayerNorm without affine, biased variance, eps_ln.
+ *   x [L_pad][D] fp32 -> xm [L_pad][D] bf16 (padding rows written as 0). */
+int h3_adaln_norm_modulate(const h3_dims* dims, const h3_ranges* ranges, const float* x, const float* mod,
+                           int branch, h3_bf16* xm, void* stream);
+
+/* A4 + A5.  [q | k | v] = xm * Wqkv^T (Wqkv [3I][D]); with
+ * H3_QK_NORM_ROPE_IN_QKV, every 128-wide head of q and k is RMS-normalised
+ * (eps_qk) and scaled by qn_w / kn_w [128], then rotated by the 3-D RoPE:
+ * head_dim splits into t | h | w sections (rope_t, rope_h, rope_w); pair
+ * (2i, 2i+1) of a section of width d turns by pos_axis * theta^(-2i/d)
+ * ([shouss] §3.2: per-head RMSNorm then positional encoding; [gojay] §7.4).
+ *   pos [L_pad][3] fp32;  q, k, v out: head-major [H][L_pad][128] bf16. */
+int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* xm, const h3_bf16* Wqkv,
+                        const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags, h3_bf16* q,
+                        h3_bf16* k, h3_bf16* v, void* stream);
+
+/* A6.  o = softmax(q k^T / sqrt(128)) v per head over all L valid tokens,
+ * non-causal; keys >= L are masked ([shouss] §5).  q, k, v: head-major
+ * [H][L_pad][128] bf16 as written by h3_qkv_qknorm_mrope (flags must carry
+ * H3_QK_NORM_ROPE_IN_QKV; qn_w, kn_w and pos are then unused and may be NULL).
+ *   o [L_pad][H*128] bf16, token-major; rows >= L written as 0. */
+int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q, const h3_bf16* k,
+                 const h3_bf16* v, const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
+                 h3_bf16* o, void* stream);
+
+/* A7.  x[r] += gate_m[branch] (.) (o * Wo^T)[r] for valid rows r, m = modality
+ * of r ([shouss] §3: shared attention + modality gate + residual).
+ *   x [L_pad][D] fp32 in/out; o [L_pad][I] bf16; Wo [D][I] bf16. */
+int h3_gated_residual(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* o,
+                      const h3_bf16* Wo, const float* mod, int branch, void* stream);
+
+/* Bytes of the h3_ffn_swiglu workspace: L_pad * F * sizeof(bf16). */
+size_t h3_ffn_workspace_bytes(const h3_dims* dims, int L_pad);
+
+/* A9.  h = SiLU(xm Wg^T) (.) (xm Wu^T) into ws, then
+ * x[r] += gate_mlp_m (.) (h Wd^T)[r] ([shouss] §3, §3.2).
+ *   Wgu [2F][D] bf16 = [gate rows; up rows]; Wd [D][F] bf16;
+ *   ws  caller-owned scratch of h3_ffn_workspace_bytes() bytes. */
+int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* xm,
+                  const h3_bf16* Wgu, const h3_bf16* Wd, const float* mod, h3_bf16* ws, void* stream);
+
+/* A10 (a reading: the pages say only that the output layers are
+ * modality-specific, [gojay] §5).  Non-affine LayerNorm of x into hn, then
+ * v_video = unpatchify(hn_video * W_vhead^T) [T][Hl][Wl][C_lat] fp32 and
+ * v_audio = hn_audio * W_ahead^T [audio_channels][n_audio][C_audio] fp32.
+ *   W_vhead [4*C_lat][D], W_ahead [C_audio][D] bf16; hn [L_pad][D] bf16 scratch. */
+int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
+                   const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
+                   int C_audio, h3_bf16* hn, float* v_video, float* v_audio, void* stream);
+
+/* A11.  lat[i] += (sigma_next - sigma) * vel[i] for i < n: one Euler step of
+ * the rectified-flow ODE on a generation target (x0 = x - sigma v;
+ * [shouss] §5, §6).  lat, vel: fp32 device arrays of n elements. */
+int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream);
+
+/* Synchronise `stream`, then report (and clear) the device error word that
+ * bounded device-side waits set when they give up.  *code_out = 0 when no
+ * wait failed.  Returns H3_ERR_TIMEOUT if one did, H3_ERR_CUDA on a CUDA
+ * error, else H3_OK. */
+int h3_device_status(void* stream, int* code_out);
+
+/* Set the time limit (nanoseconds, > 0) of every device-side wait for
+ * kernels launched afterwards on the current device (default 2 s). */
+int h3_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3_H */

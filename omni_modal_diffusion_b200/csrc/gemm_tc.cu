@@ -1,0 +1,408 @@
+// Persistent tcgen05 GEMM, out = A[M,K] * B[N,K]^T (bf16 in, fp32 accumulate
+// in TMEM), with the block's fused epilogues:
+//   - input projections into the fp32 residual stream,
+//   - modality-gated residual add (attention out-projection, FFN down),
+//   - SiLU(gate) * up (FFN gate/up),
+//   - per-head Q/K RMSNorm + 3-D RoPE with a head-major scatter (QKV),
+//   - the video head's inverse patchify gather.
+// Block structure per "MiniMax-H3: native joint audio-video generation"
+// (note.shouss.top) §3 and §3.2; patch layout per "MiniMax-H3 paper reading"
+// (gojay.top) §7.3.
+//
+// CTA = 6 warps.  Warp 0: TMA producer (one thread).  Warp 1: TMEM owner and
+// MMA issuer (one thread).  Warps 2-5: epilogue, one accumulator row per
+// thread (warp w may read TMEM lanes 32*(w%4) .. +31).  Tiles are 128 x 256
+// with a 64-deep K step, 4 shared-memory stages (48 KB each) and two TMEM
+// accumulators (2 x 256 columns) so the epilogue of one tile overlaps the
+// MMAs of the next.
+#include "h3_internal.cuh"
+#include "ptx.cuh"
+
+namespace h3 {
+
+namespace gemm_detail {
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
+
+__device__ __forceinline__ int modality_of(int row, const GemmEpilogue& e) {
+#pragma unroll
+  for (int m = 0; m < 3; ++m)
+    if (row >= e.rstart[m] && row < e.rstart[m] + e.rcount[m]) return m;
+  return -1;
+}
+
+__device__ __forceinline__ void ld_chunk(uint32_t taddr, float* v) {
+  tmem_ld32(taddr, reinterpret_cast<uint32_t*>(v));
+}
+
+// ------------------------------------------------------------ epilogues
+__device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb, int m, int n0) {
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    const int nc = n0 + c * 32;
+    if (nc >= e.N) break;  // uniform across the CTA
+    float v[32];
+    ld_chunk(tb + c * 32, v);
+    tmem_wait_ld();
+    if (m < e.M) {
+      float* dst = static_cast<float*>(e.out) + (long)(e.row_off + m) * e.ldo + nc;
+      if (nc + 32 <= e.N) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      } else {
+        for (int j = 0; j < 32 && nc + j < e.N; ++j) dst[j] = v[j];
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_gated_resid(const GemmEpilogue& e, uint32_t tb, int m, int n0) {
+  const int row = e.row_off + m;
+  const int mod_id = (m < e.M) ? modality_of(row, e) : -1;
+  const float* gate = e.mod + (long)((mod_id < 0 ? 0 : mod_id) * 6 + e.gate_slot) * e.D;
+  float* xrow = static_cast<float*>(e.out) + (long)row * e.ldo;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    const int nc = n0 + c * 32;
+    if (nc >= e.N) break;
+    float v[32];
+    ld_chunk(tb + c * 32, v);
+    tmem_wait_ld();
+    if (mod_id >= 0) {
+      if (nc + 32 <= e.N) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          float4 x = *reinterpret_cast<const float4*>(xrow + nc + j);
+          const float4 g = __ldg(reinterpret_cast<const float4*>(gate + nc + j));
+          x.x = fmaf(g.x, v[j], x.x);
+          x.y = fmaf(g.y, v[j + 1], x.y);
+          x.z = fmaf(g.z, v[j + 2], x.z);
+          x.w = fmaf(g.w, v[j + 3], x.w);
+          *reinterpret_cast<float4*>(xrow + nc + j) = x;
+        }
+      } else {
+        for (int j = 0; j < 32 && nc + j < e.N; ++j) xrow[nc + j] = fmaf(gate[nc + j], v[j], xrow[nc + j]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_swiglu(const GemmEpilogue& e, uint32_t tb, int m, int nt) {
+  // columns [0,128) of the accumulator hold gate, [128,256) hold up, for
+  // output columns nt*128 + [0,128)
+  bf16* dst = static_cast<bf16*>(e.out) + (long)m * e.ldo + (long)nt * 128;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    float g[32], u[32];
+    ld_chunk(tb + c * 32, g);
+    ld_chunk(tb + 128 + c * 32, u);
+    tmem_wait_ld();
+    if (m < e.M) {
+      uint32_t packed[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float h0 = g[j] / (1.0f + __expf(-g[j])) * u[j];
+        const float h1 = g[j + 1] / (1.0f + __expf(-g[j + 1])) * u[j + 1];
+        packed[j / 2] = pack_bf16x2(h0, h1);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; j += 4)
+        *reinterpret_cast<uint4*>(dst + c * 32 + j * 2) =
+            make_uint4(packed[j], packed[j + 1], packed[j + 2], packed[j + 3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int m, int n0, const float* freq,
+                                        const uint8_t* axis_of_pair) {
+  float p3[3] = {0.f, 0.f, 0.f};
+  if (m < e.L_pad) {
+    p3[0] = e.pos[(long)m * 3 + 0];
+    p3[1] = e.pos[(long)m * 3 + 1];
+    p3[2] = e.pos[(long)m * 3 + 2];
+  }
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    const int n = n0 + half * 128;
+    if (n >= e.N) break;  // uniform
+    const int part = n / e.I;
+    const int h = (n % e.I) / 128;
+    float v[128];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ld_chunk(tb + half * 128 + c * 32, v + c * 32);
+    tmem_wait_ld();
+    if (part < 2) {
+      float ss = 0.f;
+#pragma unroll
+      for (int d = 0; d < 128; ++d) ss = fmaf(v[d], v[d], ss);
+      const float inv = rsqrtf(ss * (1.0f / 128.0f) + e.eps_qk);
+      const bf16* w = part == 0 ? e.qn_w : e.kn_w;
+#pragma unroll
+      for (int d = 0; d < 128; d += 8) {
+        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w + d));
+        const bf16* wb = reinterpret_cast<const bf16*>(&wv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[d + j] = v[d + j] * inv * __bfloat162float(wb[j]);
+      }
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const int ax = axis_of_pair[i];
+        const float pa = ax == 0 ? p3[0] : (ax == 1 ? p3[1] : p3[2]);
+        float s, c;
+        sincosf(pa * freq[i], &s, &c);
+        const float a = v[2 * i], b = v[2 * i + 1];
+        v[2 * i] = a * c - b * s;
+        v[2 * i + 1] = a * s + b * c;
+      }
+    }
+    if (m < e.M) {
+      bf16* base = part == 0 ? e.q : (part == 1 ? e.k : e.v);
+      bf16* dst = base + ((long)h * e.L_pad + m) * 128;
+#pragma unroll
+      for (int d = 0; d < 128; d += 8) {
+        uint4 o;
+        o.x = pack_bf16x2(v[d], v[d + 1]);
+        o.y = pack_bf16x2(v[d + 2], v[d + 3]);
+        o.z = pack_bf16x2(v[d + 4], v[d + 5]);
+        o.w = pack_bf16x2(v[d + 6], v[d + 7]);
+        *reinterpret_cast<uint4*>(dst + d) = o;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_unpatch(const GemmEpilogue& e, uint32_t tb, int m, int n0) {
+  const int C = e.C_lat;
+  const int t = m / (e.Ht * e.Wt), i = (m / e.Wt) % e.Ht, j = m % e.Wt;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    const int nc = n0 + c * 32;
+    if (nc >= e.N) break;
+    float v[32];
+    ld_chunk(tb + c * 32, v);
+    tmem_wait_ld();
+    if (m < e.M) {
+      for (int jj = 0; jj < 32 && nc + jj < e.N; ++jj) {
+        const int f = nc + jj;
+        const int ph = f / (2 * C), pw = (f / C) % 2, ch = f % C;
+        const long dst = (((long)t * (2 * e.Ht) + 2 * i + ph) * (2 * e.Wt) + 2 * j + pw) * C + ch;
+        static_cast<float*>(e.out)[dst] = v[jj];
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmProblem p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  float* freq = reinterpret_cast<float*>(tmem_slot + 4);
+  uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const GemmEpilogue& e = p.epi;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (e.mode == EPI_QKV && threadIdx.x >= 64 && threadIdx.x < 128) {
+    // rotation frequency of each of the 64 pairs: section t | h | w, pair i
+    // of a section of width d turns by theta^(-2i/d) per unit position
+    const int i = threadIdx.x - 64;
+    const int pt = e.rope_t / 2, ph = e.rope_h / 2;
+    int ax, i_sec, d_sec;
+    if (i < pt) { ax = 0; i_sec = i; d_sec = e.rope_t; }
+    else if (i < pt + ph) { ax = 1; i_sec = i - pt; d_sec = e.rope_h; }
+    else { ax = 2; i_sec = i - pt - ph; d_sec = e.rope_w; }
+    freq[i] = powf(e.theta, -2.0f * (float)i_sec / (float)d_sec);
+    axis_of_pair[i] = (uint8_t)ax;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_tiles = (p.M + BM - 1) / BM;
+  const int num_tiles = m_tiles * p.n_tiles;
+  const int num_kb = (p.K + BK - 1) / BK;
+  const bool swiglu = e.mode == EPI_SWIGLU;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int mt = t % m_tiles, nt = t / m_tiles;
+        const int b0 = nt * (swiglu ? 128 : 256);
+        const int b1 = b0 + p.b_second_half_off;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(smA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, mt * BM);
+          tma_load_2d(smB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * BK, b0);
+          tma_load_2d(smB + stage * B_STAGE_BYTES + B_STAGE_BYTES / 2, &tmB, &full[stage], kb * BK, b1);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smA + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(smB + stage * B_STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int mt = t % m_tiles, nt = t / m_tiles;
+      bool ok = mbar_wait(&tfull[acc], acc_phase);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int m = mt * BM + row_in_tile;
+      switch (e.mode) {
+        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN); break;
+        case EPI_GATED_RESID: epi_gated_resid(e, tb, m, nt * BN); break;
+        case EPI_SWIGLU: epi_swiglu(e, tb, m, nt); break;
+        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair); break;
+        case EPI_UNPATCH: epi_unpatch(e, tb, m, nt * BN); break;
+        default: break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+}  // namespace gemm_detail
+using namespace gemm_detail;
+
+// 2-D bf16 tensor map with 64-element (128-byte) inner boxes and 128-byte
+// swizzle; out-of-range elements read as zero.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
+  if (p.M <= 0) return cudaSuccess;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t err = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_detail::SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    attr_set = true;
+  }
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_bf16(&tmA, p.A, (uint64_t)p.M, (uint64_t)p.K, (uint64_t)p.lda, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tmB, p.B, (uint64_t)p.N_b_rows, (uint64_t)p.K, (uint64_t)p.ldb, 128))
+    return cudaErrorInvalidValue;
+  const int m_tiles = (p.M + gemm_detail::BM - 1) / gemm_detail::BM;
+  const int tiles = m_tiles * p.n_tiles;
+  const int grid = tiles < num_sms() ? tiles : num_sms();
+  gemm_tc_kernel<<<grid, gemm_detail::NUM_THREADS, gemm_detail::SMEM_BYTES, stream>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace h3

@@ -1,0 +1,425 @@
+// C ABI of the H3-Omni block step (declarations and contracts: include/h3.h).
+// Argument validation happens here, before any launch; the kernels live in
+// the files included below (one translation unit, so the device error word
+// and wait limit are shared by every kernel without relocatable device code).
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/h3.h"
+#include "elementwise.cu"
+#include "gemm_tc.cu"
+#include "attention_tc.cu"
+
+using namespace h3;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = 0;
+  return H3_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(H3_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define H3_REQUIRE_PTR(p)                                                   \
+  do {                                                                      \
+    if (!(p)) return fail(H3_ERR_NULL, "%s: argument '%s' is NULL", __func__, #p); \
+    if (!aligned16(p)) return fail(H3_ERR_ALIGN, "%s: argument '%s' is not 16-byte aligned", __func__, #p); \
+  } while (0)
+
+int check_dims(const h3_dims* d, const char* fn) {
+  if (!d) return fail(H3_ERR_NULL, "%s: dims is NULL", fn);
+  if (d->head_dim != 128) return fail(H3_ERR_UNSUPPORTED, "%s: head_dim must be 128 (got %d)", fn, d->head_dim);
+  if (d->H <= 0 || d->I != d->H * d->head_dim)
+    return fail(H3_ERR_SHAPE, "%s: I (%d) must equal H (%d) * head_dim", fn, d->I, d->H);
+  if (d->D <= 0 || d->D % 64 != 0 || d->D > 8192)
+    return fail(H3_ERR_UNSUPPORTED, "%s: D must be a positive multiple of 64, at most 8192 (got %d)", fn, d->D);
+  if (d->F <= 0 || d->F % 128 != 0)
+    return fail(H3_ERR_UNSUPPORTED, "%s: F must be a positive multiple of 128 (got %d)", fn, d->F);
+  if (d->rope_t < 0 || d->rope_h < 0 || d->rope_w < 0 || (d->rope_t | d->rope_h | d->rope_w) & 1 ||
+      d->rope_t + d->rope_h + d->rope_w != d->head_dim)
+    return fail(H3_ERR_SHAPE, "%s: rope_t + rope_h + rope_w must equal head_dim, each even", fn);
+  if (!(d->theta > 0.f) || !(d->eps_ln > 0.f) || !(d->eps_qk > 0.f))
+    return fail(H3_ERR_SHAPE, "%s: theta, eps_ln, eps_qk must be positive", fn);
+  return H3_OK;
+}
+
+int check_ranges(const h3_ranges* r, const char* fn) {
+  if (!r) return fail(H3_ERR_NULL, "%s: ranges is NULL", fn);
+  if (r->L <= 0) return fail(H3_ERR_SHAPE, "%s: L must be positive (got %d)", fn, r->L);
+  if (r->L_pad % 128 != 0 || r->L_pad < r->L || r->L_pad - r->L >= 128)
+    return fail(H3_ERR_SHAPE, "%s: L_pad (%d) must be L (%d) rounded up to a multiple of 128", fn, r->L_pad, r->L);
+  long total = 0;
+  for (int m = 0; m < 3; ++m) {
+    if (r->start[m] < 0 || r->count[m] < 0 || (long)r->start[m] + r->count[m] > r->L)
+      return fail(H3_ERR_SHAPE, "%s: range %d [%d, +%d) outside [0, L)", fn, m, r->start[m], r->count[m]);
+    total += r->count[m];
+    for (int n = 0; n < m; ++n) {
+      const long a0 = r->start[m], a1 = a0 + r->count[m], b0 = r->start[n], b1 = b0 + r->count[n];
+      if (r->count[m] > 0 && r->count[n] > 0 && a0 < b1 && b0 < a1)
+        return fail(H3_ERR_SHAPE, "%s: ranges %d and %d overlap", fn, n, m);
+    }
+  }
+  if (total != r->L) return fail(H3_ERR_SHAPE, "%s: ranges cover %ld rows, L is %d", fn, total, r->L);
+  return H3_OK;
+}
+
+#define H3_CHECK(expr)          \
+  do {                          \
+    int _rc = (expr);           \
+    if (_rc != H3_OK) return _rc; \
+  } while (0)
+
+GemmProblem gemm_base(const void* A, long lda, int M, int K, const void* B, long ldb, int N_b_rows, int n_tiles) {
+  GemmProblem p;
+  memset(&p, 0, sizeof(p));
+  p.A = A;
+  p.lda = lda;
+  p.B = B;
+  p.ldb = ldb;
+  p.N_b_rows = N_b_rows;
+  p.M = M;
+  p.K = K;
+  p.n_tiles = n_tiles;
+  p.b_second_half_off = 128;
+  return p;
+}
+
+void set_ranges(GemmEpilogue& e, const h3_ranges* r) {
+  for (int m = 0; m < 3; ++m) {
+    e.rstart[m] = r->start[m];
+    e.rcount[m] = r->count[m];
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* h3_last_error(void) { return g_err; }
+
+int h3_version(void) { return 100; }
+
+int h3_make_ranges(int n_text, int n_audio_tokens, int n_video_tokens, h3_ranges* out) {
+  if (!out) return fail(H3_ERR_NULL, "h3_make_ranges: out is NULL");
+  if (n_text < 0 || n_audio_tokens < 0 || n_video_tokens < 0)
+    return fail(H3_ERR_SHAPE, "h3_make_ranges: negative token count");
+  const long L = (long)n_text + n_audio_tokens + n_video_tokens;
+  if (L <= 0 || L > (1L << 30)) return fail(H3_ERR_SHAPE, "h3_make_ranges: L = %ld out of range", L);
+  out->start[H3_TEXT] = 0;
+  out->count[H3_TEXT] = n_text;
+  out->start[H3_AUDIO] = n_text;
+  out->count[H3_AUDIO] = n_audio_tokens;
+  out->start[H3_VIDEO] = n_text + n_audio_tokens;
+  out->count[H3_VIDEO] = n_video_tokens;
+  out->L = (int)L;
+  out->L_pad = (int)((L + 127) / 128 * 128);
+  return ok();
+}
+
+int h3_sigma_schedule(int n_steps, float shift, float* out) {
+  if (!out) return fail(H3_ERR_NULL, "h3_sigma_schedule: out is NULL");
+  if (n_steps <= 0 || !(shift > 0.f)) return fail(H3_ERR_SHAPE, "h3_sigma_schedule: n_steps > 0 and shift > 0 required");
+  for (int i = 0; i <= n_steps; ++i) {
+    const double s = 1.0 - (double)i / n_steps;
+    out[i] = (float)(shift * s / (1.0 + (shift - 1.0) * s));
+  }
+  return ok();
+}
+
+int h3_embed_pack(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* text, int D_text,
+                  const h3_bf16* video, int T, int Hl, int Wl, int C_lat, const h3_bf16* audio,
+                  int audio_channels, int n_audio, int C_audio, const h3_bf16* W_text, const h3_bf16* W_vid,
+                  const h3_bf16* W_aud, h3_bf16* patches, float* x_out, float* pos_out, uint8_t* mod_out,
+                  void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  const int nt = ranges->count[H3_TEXT], na = ranges->count[H3_AUDIO], nv = ranges->count[H3_VIDEO];
+  if (T < 0 || Hl < 0 || Wl < 0 || (Hl & 1) || (Wl & 1))
+    return fail(H3_ERR_SHAPE, "%s: video latent T, Hl, Wl must be >= 0 with Hl, Wl even", __func__);
+  if ((long)T * (Hl / 2) * (Wl / 2) != nv)
+    return fail(H3_ERR_SHAPE, "%s: count[VIDEO] (%d) != T*(Hl/2)*(Wl/2) (%ld)", __func__, nv, (long)T * (Hl / 2) * (Wl / 2));
+  if (audio_channels < 0 || n_audio < 0 || (long)audio_channels * n_audio != na)
+    return fail(H3_ERR_SHAPE, "%s: count[AUDIO] (%d) != audio_channels*n_audio", __func__, na);
+  if (nt > 0 && (D_text <= 0 || D_text % 8))
+    return fail(H3_ERR_UNSUPPORTED, "%s: D_text must be a positive multiple of 8", __func__);
+  if (nv > 0 && (C_lat <= 0 || C_lat % 4))
+    return fail(H3_ERR_UNSUPPORTED, "%s: C_lat must be a positive multiple of 4", __func__);
+  if (na > 0 && (C_audio <= 0 || C_audio % 8))
+    return fail(H3_ERR_UNSUPPORTED, "%s: C_audio must be a positive multiple of 8", __func__);
+  H3_REQUIRE_PTR(x_out);
+  H3_REQUIRE_PTR(pos_out);
+  H3_REQUIRE_PTR(mod_out);
+  if (nt > 0) { H3_REQUIRE_PTR(text); H3_REQUIRE_PTR(W_text); }
+  if (na > 0) { H3_REQUIRE_PTR(audio); H3_REQUIRE_PTR(W_aud); }
+  if (nv > 0) { H3_REQUIRE_PTR(video); H3_REQUIRE_PTR(W_vid); H3_REQUIRE_PTR(patches); }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int D = dims->D;
+  cudaError_t e = launch_pack(reinterpret_cast<const bf16*>(video), T, Hl, Wl, C_lat, n_audio, audio_channels,
+                              ranges->start, ranges->count, ranges->L, ranges->L_pad, reinterpret_cast<bf16*>(patches),
+                              pos_out, mod_out, x_out, D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "h3_embed_pack: pack");
+  struct Src { const void* A; int K; const void* W; int mod; } srcs[3] = {
+      {text, D_text, W_text, H3_TEXT}, {audio, C_audio, W_aud, H3_AUDIO}, {patches, 4 * C_lat, W_vid, H3_VIDEO}};
+  for (const Src& s : srcs) {
+    const int M = ranges->count[s.mod];
+    if (M == 0) continue;
+    GemmProblem p = gemm_base(s.A, s.K, M, s.K, s.W, s.K, D, (D + 255) / 256);
+    p.epi.mode = EPI_STORE_F32;
+    p.epi.M = M;
+    p.epi.N = D;
+    p.epi.row_off = ranges->start[s.mod];
+    p.epi.ldo = D;
+    p.epi.out = x_out;
+    e = launch_gemm(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "h3_embed_pack: input projection");
+  }
+  return ok();
+}
+
+int h3_adaln_norm_modulate(const h3_dims* dims, const h3_ranges* ranges, const float* x, const float* mod,
+                           int branch, h3_bf16* xm, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  if (branch != H3_MSA && branch != H3_MLP) return fail(H3_ERR_SHAPE, "%s: branch must be H3_MSA or H3_MLP", __func__);
+  H3_REQUIRE_PTR(x);
+  H3_REQUIRE_PTR(mod);
+  H3_REQUIRE_PTR(xm);
+  cudaError_t e = launch_ln_modulate(x, mod, branch, ranges->start, ranges->count, ranges->L, ranges->L_pad, dims->D,
+                                     dims->eps_ln, reinterpret_cast<bf16*>(xm), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_adaln_norm_modulate");
+  return ok();
+}
+
+int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* xm, const h3_bf16* Wqkv,
+                        const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags, h3_bf16* q,
+                        h3_bf16* k, h3_bf16* v, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
+    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  H3_REQUIRE_PTR(xm);
+  H3_REQUIRE_PTR(Wqkv);
+  H3_REQUIRE_PTR(qn_w);
+  H3_REQUIRE_PTR(kn_w);
+  H3_REQUIRE_PTR(pos);
+  H3_REQUIRE_PTR(q);
+  H3_REQUIRE_PTR(k);
+  H3_REQUIRE_PTR(v);
+  const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
+  GemmProblem p = gemm_base(xm, D, Lp, D, Wqkv, D, 3 * I, (3 * I + 255) / 256);
+  GemmEpilogue& ep = p.epi;
+  ep.mode = EPI_QKV;
+  ep.M = Lp;
+  ep.N = 3 * I;
+  set_ranges(ep, ranges);
+  ep.q = reinterpret_cast<bf16*>(q);
+  ep.k = reinterpret_cast<bf16*>(k);
+  ep.v = reinterpret_cast<bf16*>(v);
+  ep.qn_w = reinterpret_cast<const bf16*>(qn_w);
+  ep.kn_w = reinterpret_cast<const bf16*>(kn_w);
+  ep.pos = pos;
+  ep.L_pad = Lp;
+  ep.I = I;
+  ep.rope_t = dims->rope_t;
+  ep.rope_h = dims->rope_h;
+  ep.rope_w = dims->rope_w;
+  ep.theta = dims->theta;
+  ep.eps_qk = dims->eps_qk;
+  cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_qkv_qknorm_mrope");
+  return ok();
+}
+
+int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q, const h3_bf16* k,
+                 const h3_bf16* v, const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
+                 h3_bf16* o, void* stream) {
+  (void)qn_w;
+  (void)kn_w;
+  (void)pos;
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
+    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  H3_REQUIRE_PTR(q);
+  H3_REQUIRE_PTR(k);
+  H3_REQUIRE_PTR(v);
+  H3_REQUIRE_PTR(o);
+  AttnProblem p;
+  p.q = reinterpret_cast<const bf16*>(q);
+  p.k = reinterpret_cast<const bf16*>(k);
+  p.v = reinterpret_cast<const bf16*>(v);
+  p.o = reinterpret_cast<bf16*>(o);
+  p.H = dims->H;
+  p.L = ranges->L;
+  p.L_pad = ranges->L_pad;
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->head_dim));
+  cudaError_t e = launch_attention(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_attention");
+  return ok();
+}
+
+int h3_gated_residual(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* o,
+                      const h3_bf16* Wo, const float* mod, int branch, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  if (branch != H3_MSA && branch != H3_MLP) return fail(H3_ERR_SHAPE, "%s: branch must be H3_MSA or H3_MLP", __func__);
+  H3_REQUIRE_PTR(x);
+  H3_REQUIRE_PTR(o);
+  H3_REQUIRE_PTR(Wo);
+  H3_REQUIRE_PTR(mod);
+  const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
+  GemmProblem p = gemm_base(o, I, Lp, I, Wo, I, D, (D + 255) / 256);
+  p.epi.mode = EPI_GATED_RESID;
+  p.epi.M = Lp;
+  p.epi.N = D;
+  p.epi.ldo = D;
+  p.epi.out = x;
+  set_ranges(p.epi, ranges);
+  p.epi.mod = mod;
+  p.epi.gate_slot = 3 * branch + 2;
+  p.epi.D = D;
+  cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_gated_residual");
+  return ok();
+}
+
+size_t h3_ffn_workspace_bytes(const h3_dims* dims, int L_pad) {
+  if (!dims || L_pad <= 0 || dims->F <= 0) return 0;
+  return (size_t)L_pad * (size_t)dims->F * 2;
+}
+
+int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* xm,
+                  const h3_bf16* Wgu, const h3_bf16* Wd, const float* mod, h3_bf16* ws, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  H3_REQUIRE_PTR(x);
+  H3_REQUIRE_PTR(xm);
+  H3_REQUIRE_PTR(Wgu);
+  H3_REQUIRE_PTR(Wd);
+  H3_REQUIRE_PTR(mod);
+  H3_REQUIRE_PTR(ws);
+  const int D = dims->D, F = dims->F, Lp = ranges->L_pad;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GemmProblem p1 = gemm_base(xm, D, Lp, D, Wgu, D, 2 * F, F / 128);
+  p1.b_second_half_off = F;
+  p1.epi.mode = EPI_SWIGLU;
+  p1.epi.M = Lp;
+  p1.epi.N = F;
+  p1.epi.ldo = F;
+  p1.epi.out = ws;
+  cudaError_t e = launch_gemm(p1, st);
+  if (e != cudaSuccess) return cuda_fail(e, "h3_ffn_swiglu: gate/up");
+  GemmProblem p2 = gemm_base(ws, F, Lp, F, Wd, F, D, (D + 255) / 256);
+  p2.epi.mode = EPI_GATED_RESID;
+  p2.epi.M = Lp;
+  p2.epi.N = D;
+  p2.epi.ldo = D;
+  p2.epi.out = x;
+  set_ranges(p2.epi, ranges);
+  p2.epi.mod = mod;
+  p2.epi.gate_slot = 5;
+  p2.epi.D = D;
+  e = launch_gemm(p2, st);
+  if (e != cudaSuccess) return cuda_fail(e, "h3_ffn_swiglu: down");
+  return ok();
+}
+
+int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
+                   const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
+                   int C_audio, h3_bf16* hn, float* v_video, float* v_audio, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  const int na = ranges->count[H3_AUDIO], nv = ranges->count[H3_VIDEO];
+  if (T < 0 || (Hl & 1) || (Wl & 1) || (long)T * (Hl / 2) * (Wl / 2) != nv)
+    return fail(H3_ERR_SHAPE, "%s: count[VIDEO] != T*(Hl/2)*(Wl/2)", __func__);
+  if ((long)audio_channels * n_audio != na) return fail(H3_ERR_SHAPE, "%s: count[AUDIO] != channels*n_audio", __func__);
+  if (nv > 0 && (C_lat <= 0 || C_lat % 4)) return fail(H3_ERR_UNSUPPORTED, "%s: C_lat must be a multiple of 4", __func__);
+  if (na > 0 && (C_audio <= 0 || C_audio % 4)) return fail(H3_ERR_UNSUPPORTED, "%s: C_audio must be a multiple of 4", __func__);
+  H3_REQUIRE_PTR(x);
+  H3_REQUIRE_PTR(hn);
+  if (nv > 0) { H3_REQUIRE_PTR(W_vhead); H3_REQUIRE_PTR(v_video); }
+  if (na > 0) { H3_REQUIRE_PTR(W_ahead); H3_REQUIRE_PTR(v_audio); }
+  const int D = dims->D;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_ln_modulate(x, nullptr, 0, ranges->start, ranges->count, ranges->L, ranges->L_pad, D,
+                                     dims->eps_ln, reinterpret_cast<bf16*>(hn), st);
+  if (e != cudaSuccess) return cuda_fail(e, "h3_head_unpack: norm");
+  if (nv > 0) {
+    const h3_bf16* A = hn + (size_t)ranges->start[H3_VIDEO] * D;
+    GemmProblem p = gemm_base(A, D, nv, D, W_vhead, D, 4 * C_lat, (4 * C_lat + 255) / 256);
+    p.epi.mode = EPI_UNPATCH;
+    p.epi.M = nv;
+    p.epi.N = 4 * C_lat;
+    p.epi.out = v_video;
+    p.epi.Ht = Hl / 2;
+    p.epi.Wt = Wl / 2;
+    p.epi.C_lat = C_lat;
+    e = launch_gemm(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "h3_head_unpack: video head");
+  }
+  if (na > 0) {
+    const h3_bf16* A = hn + (size_t)ranges->start[H3_AUDIO] * D;
+    GemmProblem p = gemm_base(A, D, na, D, W_ahead, D, C_audio, (C_audio + 255) / 256);
+    p.epi.mode = EPI_STORE_F32;
+    p.epi.M = na;
+    p.epi.N = C_audio;
+    p.epi.ldo = C_audio;
+    p.epi.out = v_audio;
+    e = launch_gemm(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "h3_head_unpack: audio head");
+  }
+  return ok();
+}
+
+int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream) {
+  if (n < 0) return fail(H3_ERR_SHAPE, "h3_euler_step: n < 0");
+  if (n == 0) return ok();
+  H3_REQUIRE_PTR(lat);
+  H3_REQUIRE_PTR(vel);
+  cudaError_t e = launch_euler(lat, vel, (long long)n, sigma_next - sigma, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_euler_step");
+  return ok();
+}
+
+int h3_device_status(void* stream, int* code_out) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: synchronize");
+  int code = 0;
+  e = cudaMemcpyFromSymbol(&code, g_h3_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: read");
+  if (code != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_h3_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: clear");
+  }
+  if (code_out) *code_out = code;
+  if (code != 0) return fail(H3_ERR_TIMEOUT, "h3_device_status: a device-side wait gave up (code %d)", code);
+  return ok();
+}
+
+int h3_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) return fail(H3_ERR_SHAPE, "h3_set_wait_limit_ns: limit must be > 0");
+  unsigned long long v = ns;
+  cudaError_t e = cudaMemcpyToSymbol(g_h3_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_set_wait_limit_ns");
+  return ok();
+}
+
+}  // extern "C"

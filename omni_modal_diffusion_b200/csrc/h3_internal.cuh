@@ -1,0 +1,82 @@
+// Internal launch interfaces shared by the C-ABI layer and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace h3 {
+
+typedef __nv_bfloat16 bf16;
+
+// Epilogue variants of the tensor-core GEMM (out = A[M,K] * B[N,K]^T).
+enum EpiMode : int {
+  EPI_STORE_F32 = 0,    // out_f32[(row_off + m) * ldo + n] = acc
+  EPI_GATED_RESID = 1,  // x[(row_off + m) * ldo + n] += gate[mod(row)][n] * acc
+  EPI_SWIGLU = 2,       // ws[m * ldo + n] = bf16(SiLU(acc_gate) * acc_up)
+  EPI_QKV = 3,          // per-head Q/K RMSNorm + 3-D RoPE, head-major bf16 scatter
+  EPI_UNPATCH = 4,      // video head: acc row -> latent gather (inverse patchify), f32
+};
+
+struct GemmEpilogue {
+  int mode;
+  int M, N;          // valid output rows / columns of this GEMM
+  int row_off;       // packed-sequence row of GEMM row 0
+  long ldo;          // output row stride (elements)
+  void* out;         // EPI_STORE_F32 / EPI_GATED_RESID (x) / EPI_SWIGLU (ws) / EPI_UNPATCH
+  // modality ranges (packed rows) for gate selection
+  int rstart[3], rcount[3];
+  const float* mod;  // [3][6][D] fp32
+  int gate_slot;     // 2 (gate_msa) or 5 (gate_mlp)
+  int D;
+  // EPI_QKV
+  bf16* q;
+  bf16* k;
+  bf16* v;
+  const bf16* qn_w;
+  const bf16* kn_w;
+  const float* pos;  // [L_pad][3]
+  int L_pad, I;
+  int rope_t, rope_h, rope_w;
+  float theta, eps_qk;
+  // EPI_UNPATCH: token grid (T, Ht, Wt), latent channels
+  int Ht, Wt, C_lat;
+};
+
+struct GemmProblem {
+  const void* A;  // bf16 [M, K] row-major
+  long lda;       // elements
+  const void* B;  // bf16 [N_b, K] row-major ([out, in] weight)
+  long ldb;
+  int N_b_rows;   // rows of B (for the tensor map extent)
+  int M, K;
+  int n_tiles;    // number of 256-wide (or 128-pair for SwiGLU) column tiles
+  int b_second_half_off;  // SwiGLU: row offset of the "up" half in B (= F); else 128
+  GemmEpilogue epi;
+};
+
+// Launch one tensor-core GEMM on `stream`.  Returns a cudaError_t.
+cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream);
+
+// Attention over head-major q, k, v [H][L_pad][128] -> o [L_pad][H*128].
+struct AttnProblem {
+  const bf16* q;
+  const bf16* k;
+  const bf16* v;
+  bf16* o;
+  int H, L, L_pad;
+  float scale_log2;  // log2(e) / sqrt(head_dim)
+};
+cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream);
+
+// Memory-bound kernels.
+cudaError_t launch_pack(const bf16* video, int T, int Hl, int Wl, int C_lat, int n_audio, int audio_channels,
+                        const int* rstart, const int* rcount, int L, int L_pad, bf16* patches, float* pos,
+                        uint8_t* mod_ids, float* x, int D, cudaStream_t stream);
+cudaError_t launch_ln_modulate(const float* x, const float* mod, int branch, const int* rstart, const int* rcount,
+                               int L, int L_pad, int D, float eps, bf16* out, cudaStream_t stream);
+cudaError_t launch_euler(float* lat, const float* vel, long long n, float dsigma, cudaStream_t stream);
+
+int num_sms();
+
+}  // namespace h3

@@ -1,0 +1,198 @@
+"""Thin ctypes binding of libh3.so (include/h3.h), same names as the C ABI.
+
+Argument marshalling only: torch tensors supply device memory and the CUDA
+stream; every step of the block runs in the library's kernels.  There is no
+fallback: if the library is missing or a tensor is not a CUDA tensor of the
+expected dtype, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libh3.so")
+
+H3_OK, H3_ERR_NULL, H3_ERR_SHAPE, H3_ERR_ALIGN, H3_ERR_UNSUPPORTED, H3_ERR_CUDA, H3_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+H3_TEXT, H3_AUDIO, H3_VIDEO = 0, 1, 2
+H3_MSA, H3_MLP = 0, 1
+H3_QK_NORM_ROPE_IN_QKV = 1
+
+EXPORTS = (
+    "h3_last_error", "h3_version", "h3_make_ranges", "h3_sigma_schedule", "h3_embed_pack",
+    "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention", "h3_gated_residual",
+    "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
+    "h3_set_wait_limit_ns",
+)
+
+
+class H3Error(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"h3 status {code}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("D", ctypes.c_int), ("H", ctypes.c_int), ("head_dim", ctypes.c_int), ("I", ctypes.c_int),
+                ("F", ctypes.c_int), ("rope_t", ctypes.c_int), ("rope_h", ctypes.c_int), ("rope_w", ctypes.c_int),
+                ("theta", ctypes.c_float), ("eps_ln", ctypes.c_float), ("eps_qk", ctypes.c_float)]
+
+
+class Ranges(ctypes.Structure):
+    _fields_ = [("start", ctypes.c_int * 3), ("count", ctypes.c_int * 3), ("L", ctypes.c_int), ("L_pad", ctypes.c_int)]
+
+    def as_dict(self) -> dict:
+        return {"start": list(self.start), "count": list(self.count), "L": self.L, "L_pad": self.L_pad}
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libh3.so (raises if it is missing: there is no other code path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with python -m omni_modal_diffusion_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci, cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        pd, pr = ctypes.POINTER(Dims), ctypes.POINTER(Ranges)
+        sig = {
+            "h3_last_error": (ctypes.c_char_p, []),
+            "h3_version": (ci, []),
+            "h3_make_ranges": (ci, [ci, ci, ci, pr]),
+            "h3_sigma_schedule": (ci, [ci, cf, ctypes.POINTER(ctypes.c_float)]),
+            "h3_embed_pack": (ci, [pd, pr, vp, ci, vp, ci, ci, ci, ci, vp, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, vp]),
+            "h3_adaln_norm_modulate": (ci, [pd, pr, vp, vp, ci, vp, vp]),
+            "h3_qkv_qknorm_mrope": (ci, [pd, pr, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp]),
+            "h3_attention": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, ci, vp, vp]),
+            "h3_gated_residual": (ci, [pd, pr, vp, vp, vp, vp, ci, vp]),
+            "h3_ffn_workspace_bytes": (ctypes.c_size_t, [pd, ci]),
+            "h3_ffn_swiglu": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, vp]),
+            "h3_head_unpack": (ci, [pd, pr, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]),
+            "h3_euler_step": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp]),
+            "h3_device_status": (ci, [vp, ctypes.POINTER(ci)]),
+            "h3_set_wait_limit_ns": (ci, [ctypes.c_uint64]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != H3_OK:
+        raise H3Error(rc, lib().h3_last_error().decode())
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_dims(D, H, F, head_dim=128, rope=(32, 48, 48), theta=10000.0, eps_ln=1e-6, eps_qk=1e-6) -> Dims:
+    return Dims(D, H, head_dim, H * head_dim, F, rope[0], rope[1], rope[2], theta, eps_ln, eps_qk)
+
+
+def h3_make_ranges(n_text: int, n_audio_tokens: int, n_video_tokens: int) -> Ranges:
+    r = Ranges()
+    _check(lib().h3_make_ranges(n_text, n_audio_tokens, n_video_tokens, ctypes.byref(r)))
+    return r
+
+
+def h3_sigma_schedule(n_steps: int, shift: float) -> list[float]:
+    out = (ctypes.c_float * (n_steps + 1))()
+    _check(lib().h3_sigma_schedule(n_steps, shift, out))
+    return list(out)
+
+
+BF16, F32, U8 = torch.bfloat16, torch.float32, torch.uint8
+
+
+def h3_embed_pack(dims, ranges, text, video, audio, W_text, W_vid, W_aud, patches, x_out, pos_out, mod_out, stream=None):
+    T, Hl, Wl, C_lat = video.shape if video is not None else (0, 0, 0, 0)
+    ch, n_a, C_a = audio.shape if audio is not None else (0, 0, 0)
+    D_text = text.shape[1] if text is not None else 0
+    _check(lib().h3_embed_pack(ctypes.byref(dims), ctypes.byref(ranges), _ptr(text, BF16, "text"), D_text,
+                               _ptr(video, BF16, "video"), T, Hl, Wl, C_lat, _ptr(audio, BF16, "audio"), ch, n_a, C_a,
+                               _ptr(W_text, BF16, "W_text"), _ptr(W_vid, BF16, "W_vid"), _ptr(W_aud, BF16, "W_aud"),
+                               _ptr(patches, BF16, "patches"), _ptr(x_out, F32, "x_out"), _ptr(pos_out, F32, "pos_out"),
+                               _ptr(mod_out, U8, "mod_out"), _stream(stream)))
+
+
+def h3_adaln_norm_modulate(dims, ranges, x, mod, branch, xm, stream=None):
+    _check(lib().h3_adaln_norm_modulate(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                                        _ptr(mod, F32, "mod"), branch, _ptr(xm, BF16, "xm"), _stream(stream)))
+
+
+def h3_qkv_qknorm_mrope(dims, ranges, xm, Wqkv, qn_w, kn_w, pos, q, k, v, flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_qkv_qknorm_mrope(ctypes.byref(dims), ctypes.byref(ranges), _ptr(xm, BF16, "xm"),
+                                     _ptr(Wqkv, BF16, "Wqkv"), _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"),
+                                     _ptr(pos, F32, "pos"), flags, _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+                                     _ptr(v, BF16, "v"), _stream(stream)))
+
+
+def h3_attention(dims, ranges, q, k, v, o, qn_w=None, kn_w=None, pos=None, flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_attention(ctypes.byref(dims), ctypes.byref(ranges), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+                              _ptr(v, BF16, "v"), _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"),
+                              _ptr(pos, F32, "pos"), flags, _ptr(o, BF16, "o"), _stream(stream)))
+
+
+def h3_gated_residual(dims, ranges, x, o, Wo, mod, branch=H3_MSA, stream=None):
+    _check(lib().h3_gated_residual(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"), _ptr(o, BF16, "o"),
+                                   _ptr(Wo, BF16, "Wo"), _ptr(mod, F32, "mod"), branch, _stream(stream)))
+
+
+def h3_ffn_workspace_bytes(dims, L_pad: int) -> int:
+    return int(lib().h3_ffn_workspace_bytes(ctypes.byref(dims), L_pad))
+
+
+def h3_ffn_swiglu(dims, ranges, x, xm, Wgu, Wd, mod, ws, stream=None):
+    _check(lib().h3_ffn_swiglu(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"), _ptr(xm, BF16, "xm"),
+                               _ptr(Wgu, BF16, "Wgu"), _ptr(Wd, BF16, "Wd"), _ptr(mod, F32, "mod"),
+                               _ptr(ws, BF16, "ws"), _stream(stream)))
+
+
+def h3_head_unpack(dims, ranges, x, W_vhead, W_ahead, video_shape, audio_shape, hn, v_video, v_audio, stream=None):
+    T, Hl, Wl, C_lat = video_shape
+    ch, n_a, C_a = audio_shape
+    _check(lib().h3_head_unpack(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                                _ptr(W_vhead, BF16, "W_vhead"), _ptr(W_ahead, BF16, "W_ahead"), T, Hl, Wl, C_lat, ch,
+                                n_a, C_a, _ptr(hn, BF16, "hn"), _ptr(v_video, F32, "v_video"),
+                                _ptr(v_audio, F32, "v_audio"), _stream(stream)))
+
+
+def h3_euler_step(lat, vel, sigma: float, sigma_next: float, stream=None):
+    if lat.numel() != vel.numel():
+        raise ValueError("lat and vel sizes differ")
+    _check(lib().h3_euler_step(_ptr(lat, F32, "lat"), _ptr(vel, F32, "vel"), lat.numel(), sigma, sigma_next,
+                               _stream(stream)))
+
+
+def h3_device_status(stream=None) -> int:
+    code = ctypes.c_int(0)
+    rc = lib().h3_device_status(_stream(stream), ctypes.byref(code))
+    if rc not in (H3_OK, H3_ERR_TIMEOUT):
+        _check(rc)
+    return code.value
+
+
+def h3_set_wait_limit_ns(ns: int):
+    _check(lib().h3_set_wait_limit_ns(ns))

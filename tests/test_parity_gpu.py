@@ -1,0 +1,209 @@
+"""GPU parity: every C-ABI call against the float64 oracle on the same seeded,
+bf16-rounded inputs.  Integer/byte/index work is compared bit-exactly; floating
+point within the block tolerance (parity_util.check_close)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import h3_oracle as O
+from omni_modal_diffusion_b200 import synthetic as S
+from omni_modal_diffusion_b200 import h3
+from omni_modal_diffusion_b200.pipeline import H3BlockStep, to_dev_bf16
+
+from parity_util import RAGGED, check_close, oracle_ranges_and_pos, to_np
+
+pytestmark = pytest.mark.gpu
+
+WORKLOADS = [S.WORKLOADS["tiny"], RAGGED]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from omni_modal_diffusion_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    torch.cuda.init()
+
+
+def _setup(w):
+    inp = S.make_inputs(w)
+    st = H3BlockStep(w, weights=inp)
+    dev = st.device
+    text, video, audio = (to_dev_bf16(inp[k], dev) for k in ("text", "video", "audio"))
+    mod = torch.from_numpy(inp["mod"]).to(dev)
+    return inp, st, text, video, audio, mod
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+def test_embed_pack_bit_exact_packing_and_projection(w):
+    inp, st, text, video, audio, mod = _setup(w)
+    st.embed(text, video, audio)
+    torch.cuda.synchronize()
+    r, pos = oracle_ranges_and_pos(w)
+    assert st.ranges.as_dict() == r
+    L, Lp = r["L"], r["L_pad"]
+    # patches: an integer gather, bit-exact
+    assert np.array_equal(to_np(st.patches), O.patchify(inp["video"]))
+    # positions: fp32 of the oracle's values, bit-exact
+    assert np.array_equal(st.pos.cpu().numpy()[:L], pos.astype(np.float32))
+    assert np.all(st.pos.cpu().numpy()[L:] == 0)
+    mids = st.mod_ids.cpu().numpy()
+    assert np.array_equal(mids[:L], O.modality_of_rows(r).astype(np.uint8))
+    assert np.all(mids[L:] == 255)
+    x = to_np(st.x)
+    ref = O.embed(inp["text"], inp["video"], inp["audio"], inp["W_text"], inp["W_vid"], inp["W_aud"], r)
+    check_close(x[:L], ref, "embed x", 1e-4, 1e-5)          # fp32 accumulate of exact bf16 products
+    assert np.all(x[L:] == 0)
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+def test_block_calls_each_against_oracle(w):
+    inp, st, text, video, audio, mod = _setup(w)
+    r, pos = oracle_ranges_and_pos(w)
+    L = r["L"]
+    st.embed(text, video, audio)
+    x0 = to_np(st.x)[:L]
+    d, rg = st.dims, st.ranges
+    # A3: LN + modulate
+    h3.h3_adaln_norm_modulate(d, rg, st.x, mod, h3.H3_MSA, st.xm)
+    xm = to_np(st.xm)
+    check_close(xm[:L], O.adaln_modulate(x0, inp["mod"], r, O.MSA), "ln_modulate msa", 2e-2, 3e-3)
+    assert np.all(xm[L:] == 0)
+    # A4/A5: QKV + Q/K RMSNorm + RoPE, from the GPU's own xm
+    h3.h3_qkv_qknorm_mrope(d, rg, st.xm, st.W["Wqkv"], st.W["qn_w"], st.W["kn_w"], st.pos, st.q, st.k, st.v)
+    q_ref, k_ref, v_ref = O.qkv_qknorm_mrope(xm[:L], inp["Wqkv"], inp["qn_w"], inp["kn_w"], pos, w.H)
+    for name, g, o in (("q", st.q, q_ref), ("k", st.k, k_ref), ("v", st.v, v_ref)):
+        gg = to_np(g)[:, :L, :].transpose(1, 0, 2)
+        check_close(gg, o, name, 2e-2, 3e-3)
+    # A6: attention from the GPU's own q, k, v
+    h3.h3_attention(d, rg, st.q, st.k, st.v, st.o)
+    qg, kg, vg = (to_np(t)[:, :L, :].transpose(1, 0, 2) for t in (st.q, st.k, st.v))
+    o = to_np(st.o)
+    check_close(o[:L], O.attention(qg, kg, vg), "attention", 2e-2, 3e-3)
+    assert np.all(o[L:] == 0)
+    # A7: gated residual from the GPU's own o
+    h3.h3_gated_residual(d, rg, st.x, st.o, st.W["Wo"], mod, h3.H3_MSA)
+    x1 = to_np(st.x)[:L]
+    check_close(x1 - x0, O.gated_residual(x0, o[:L], inp["Wo"], inp["mod"], r) - x0, "gated residual delta",
+                1e-3, 1e-4)
+    # A8/A9: LN-mlp + SwiGLU FFN from the GPU's own x1
+    h3.h3_adaln_norm_modulate(d, rg, st.x, mod, h3.H3_MLP, st.xm)
+    xm2 = to_np(st.xm)[:L]
+    check_close(xm2, O.adaln_modulate(x1, inp["mod"], r, O.MLP), "ln_modulate mlp", 2e-2, 3e-3)
+    h3.h3_ffn_swiglu(d, rg, st.x, st.xm, st.W["Wgu"], st.W["Wd"], mod, st.ws)
+    x2 = to_np(st.x)[:L]
+    check_close(x2 - x1, O.ffn_swiglu(x1, xm2, inp["Wgu"], inp["Wd"], inp["mod"], r) - x1, "ffn delta")
+    assert np.all(to_np(st.x)[L:] == 0)
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+def test_block_end_to_end_against_oracle(w):
+    inp, st, text, video, audio, mod = _setup(w)
+    r, pos = oracle_ranges_and_pos(w)
+    L = r["L"]
+    st.embed(text, video, audio)
+    x0 = to_np(st.x)[:L]
+    st.block(mod)
+    x2 = to_np(st.x)[:L]
+    ref, parts = O.block_forward(x0, inp["mod"], r, pos, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"],
+                                 inp["Wgu"], inp["Wd"], w.H, return_parts=True)
+    check_close(x2, ref, "block output")
+    # The branch delta (x_out - x_in) is checked too, so that the residual
+    # cannot mask a branch error.  Its max bound follows from the bf16
+    # operands: rounding xm, q/k/v, P, o and the SwiGLU product to bf16 at
+    # exactly the points this path does, in float64 on the CPU, already gives
+    # max|err| = 0.030 * RMS(delta) on the ragged workload (mean rel 3.1e-3);
+    # 5e-2 leaves room for fp32 accumulation order and ex2.approx.
+    check_close(x2 - x0, ref - x0, "block delta", max_rel_rms=5e-2)
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+def test_head_and_euler_against_oracle(w):
+    inp, st, text, video, audio, mod = _setup(w)
+    r, _ = oracle_ranges_and_pos(w)
+    st.embed(text, video, audio)
+    st.block(mod)
+    x2 = to_np(st.x)[:r["L"]]
+    st.head()
+    t, i, j = O.token_grid(w.T_lat, w.H_lat, w.W_lat)
+    vv, va = O.head_unpack(x2, r, inp["W_vhead"], inp["W_ahead"], w.T_lat, w.H_lat, w.W_lat, w.audio_channels,
+                           w.n_audio)
+    check_close(to_np(st.v_video), vv, "video head", 2e-2, 3e-3)
+    check_close(to_np(st.v_audio), va, "audio head", 2e-2, 3e-3)
+    # Euler on each modality with its own shifted schedule
+    rng = np.random.default_rng(5)
+    lat_v = rng.standard_normal(st.v_video.shape).astype(np.float32)
+    lat_a = rng.standard_normal(st.v_audio.shape).astype(np.float32)
+    sv, sa = O.sigma_schedule(8, 12.0), O.sigma_schedule(8, 3.0)
+    gv, ga = torch.from_numpy(lat_v).cuda(), torch.from_numpy(lat_a).cuda()
+    st.euler(gv, ga, (float(sv[2]), float(sv[3])), (float(sa[2]), float(sa[3])))
+    ev = O.euler_step(lat_v, to_np(st.v_video), np.float32(sv[2]), np.float32(sv[3]))
+    ea = O.euler_step(lat_a, to_np(st.v_audio), np.float32(sa[2]), np.float32(sa[3]))
+    check_close(to_np(gv), ev, "euler video", 1e-5, 1e-6)
+    check_close(to_np(ga), ea, "euler audio", 1e-5, 1e-6)
+    # sigma 0.7 -> 0 gives the clean latent x0 = x - sigma v
+    g = torch.from_numpy(lat_v).cuda()
+    h3.h3_euler_step(g, st.v_video, 0.7, 0.0)
+    check_close(to_np(g), O.clean_latent(lat_v, to_np(st.v_video), np.float32(0.7)), "clean latent", 1e-5, 1e-6)
+
+
+def test_zero_modulation_block_is_bit_exact_identity():
+    w = S.WORKLOADS["tiny"]
+    inp, st, text, video, audio, mod = _setup(w)
+    st.embed(text, video, audio)
+    x0 = st.x.clone()
+    st.block(torch.zeros_like(mod))
+    torch.cuda.synchronize()
+    assert torch.equal(st.x, x0)
+    # gate 0 on one modality: exactly that range unchanged
+    r, _ = oracle_ranges_and_pos(w)
+    for m in range(3):
+        st.x.copy_(x0)
+        m2 = mod.clone()
+        m2[m, 2] = 0
+        m2[m, 5] = 0
+        st.block(m2)
+        torch.cuda.synchronize()
+        s, c = r["start"][m], r["count"][m]
+        assert torch.equal(st.x[s:s + c], x0[s:s + c])
+        others = [mm for mm in range(3) if mm != m]
+        for mm in others:
+            s2, c2 = r["start"][mm], r["count"][mm]
+            assert bool((st.x[s2:s2 + c2] != x0[s2:s2 + c2]).any(dim=1).all())
+
+
+def test_block_is_deterministic():
+    w = RAGGED
+    inp, st, text, video, audio, mod = _setup(w)
+    outs = []
+    for _ in range(2):
+        st.embed(text, video, audio)
+        st.block(mod)
+        st.head()
+        torch.cuda.synchronize()
+        outs.append((st.x.clone(), st.v_video.clone(), st.v_audio.clone()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_attention_single_token_and_one_tile():
+    """Edge cases: L = 1 (one key: output = v) and L = 128 (one full tile)."""
+    w = S.WORKLOADS["tiny"]
+    for L in (1, 128, 129):
+        d = h3.make_dims(w.D, w.H, w.F)
+        rg = h3.h3_make_ranges(L, 0, 0)
+        Lp = rg.L_pad
+        rng = np.random.default_rng(L)
+        qkv = [S.bf16_round(rng.standard_normal((w.H, Lp, 128)).astype(np.float32)) for _ in range(3)]
+        q, k, v = (to_dev_bf16(a, "cuda") for a in qkv)
+        o = torch.empty(Lp, w.H * 128, dtype=torch.bfloat16, device="cuda")
+        h3.h3_attention(d, rg, q, k, v, o)
+        got = to_np(o)
+        ref = O.attention(*(a[:, :L, :].transpose(1, 0, 2).astype(np.float64) for a in qkv))
+        check_close(got[:L], ref, f"attention L={L}", 2e-2, 3e-3)
+        if L == 1:
+            assert np.allclose(got[0], qkv[2][:, 0, :].reshape(-1), rtol=1e-2, atol=1e-2)
+
+
+def test_device_status_clean_after_work():
+    assert h3.h3_device_status() == 0
