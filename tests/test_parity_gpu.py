@@ -75,11 +75,13 @@ def test_block_calls_each_against_oracle(w):
     for name, g, o in (("q", st.q, q_ref), ("k", st.k, k_ref), ("v", st.v, v_ref)):
         gg = to_np(g)[:, :L, :].transpose(1, 0, 2)
         check_close(gg, o, name, 2e-2, 3e-3)
-    # A6: attention from the GPU's own q, k, v
+    # A6: attention from the GPU's own q, k, v.  Block tolerance: rounding P
+    # and o to bf16 alone (float64 emulation on the CPU) gives up to
+    # 0.024 * RMS at L = 128, so the tighter per-call bounds do not apply.
     h3.h3_attention(d, rg, st.q, st.k, st.v, st.o)
     qg, kg, vg = (to_np(t)[:, :L, :].transpose(1, 0, 2) for t in (st.q, st.k, st.v))
     o = to_np(st.o)
-    check_close(o[:L], O.attention(qg, kg, vg), "attention", 2e-2, 3e-3)
+    check_close(o[:L], O.attention(qg, kg, vg), "attention")
     assert np.all(o[L:] == 0)
     # A7: gated residual from the GPU's own o
     h3.h3_gated_residual(d, rg, st.x, st.o, st.W["Wo"], mod, h3.H3_MSA)
@@ -200,7 +202,7 @@ def test_attention_single_token_and_one_tile():
         h3.h3_attention(d, rg, q, k, v, o)
         got = to_np(o)
         ref = O.attention(*(a[:, :L, :].transpose(1, 0, 2).astype(np.float64) for a in qkv))
-        check_close(got[:L], ref, f"attention L={L}", 2e-2, 3e-3)
+        check_close(got[:L], ref, f"attention L={L}")        # block tolerance (see above)
         if L == 1:
             assert np.allclose(got[0], qkv[2][:, 0, :].reshape(-1), rtol=1e-2, atol=1e-2)
 
