@@ -166,6 +166,32 @@ size_t h3_ffn_workspace_bytes(const h3_dims* dims, int L_pad);
 int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* xm,
                   const h3_bf16* Wgu, const h3_bf16* Wd, const float* mod, h3_bf16* ws, void* stream);
 
+/* Size in bytes of the device array that h3_ffn_swiglu_noalloc uses as its
+ * workspace: 32 MiB, i.e. L_pad * F <= 16 Mi elements (at F = 14336, up to
+ * L_pad = 1152 tokens). */
+#define H3_FFN_STATIC_WS_BYTES (32u * 1024u * 1024u)
+
+/* h3_ffn_swiglu without a caller workspace; nothing is allocated.  No
+ * counterpart on the pages: this entry point exists for callers that own
+ * only their inputs and outputs and cannot obtain device memory for scratch
+ * (an operator or plugin interface that passes tensors but no workspace, a
+ * process whose device memory is all reserved by another allocator, a
+ * serving loop that must not allocate on its hot path).  Same arguments and
+ * result as h3_ffn_swiglu minus ws.
+ *   - The workspace is a fixed device array of H3_FFN_STATIC_WS_BYTES inside
+ *     the library, present on every GPU that loads it until the process
+ *     exits.  Calls with L_pad * F * 2 > H3_FFN_STATIC_WS_BYTES are rejected
+ *     with H3_ERR_SHAPE before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     calls whose kernels overlap on the GPU (other streams, other host
+ *     threads) race on it and must be serialised by the caller.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. */
+int h3_ffn_swiglu_noalloc(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* xm,
+                          const h3_bf16* Wgu, const h3_bf16* Wd, const float* mod, void* stream);
+
 /* A10 (a reading: the pages say only that the output layers are
  * modality-specific, [gojay] §5).  Non-affine LayerNorm of x into hn, then
  * v_video = unpatchify(hn_video * W_vhead^T) [T][Hl][Wl][C_lat] fp32 and

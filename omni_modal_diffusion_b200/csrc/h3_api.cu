@@ -423,3 +423,6 @@ int h3_set_wait_limit_ns(uint64_t ns) {
 }
 
 }  // extern "C"
+
+// Workspace-free variant of h3_ffn_swiglu (uses this file's checks and launcher).
+#include "h3_noalloc.cu"

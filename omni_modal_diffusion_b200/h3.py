@@ -24,8 +24,9 @@ EXPORTS = (
     "h3_last_error", "h3_version", "h3_make_ranges", "h3_sigma_schedule", "h3_embed_pack",
     "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention", "h3_gated_residual",
     "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
-    "h3_set_wait_limit_ns",
+    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc",
 )
+H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
 
 
 class H3Error(RuntimeError):
@@ -71,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "h3_gated_residual": (ci, [pd, pr, vp, vp, vp, vp, ci, vp]),
             "h3_ffn_workspace_bytes": (ctypes.c_size_t, [pd, ci]),
             "h3_ffn_swiglu": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, vp]),
+            "h3_ffn_swiglu_noalloc": (ci, [pd, pr, vp, vp, vp, vp, vp, vp]),
             "h3_head_unpack": (ci, [pd, pr, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]),
             "h3_euler_step": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp]),
             "h3_device_status": (ci, [vp, ctypes.POINTER(ci)]),
@@ -168,6 +170,13 @@ def h3_ffn_swiglu(dims, ranges, x, xm, Wgu, Wd, mod, ws, stream=None):
     _check(lib().h3_ffn_swiglu(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"), _ptr(xm, BF16, "xm"),
                                _ptr(Wgu, BF16, "Wgu"), _ptr(Wd, BF16, "Wd"), _ptr(mod, F32, "mod"),
                                _ptr(ws, BF16, "ws"), _stream(stream)))
+
+
+def h3_ffn_swiglu_noalloc(dims, ranges, x, xm, Wgu, Wd, mod, stream=None):
+    """h3_ffn_swiglu with the library's fixed device workspace (no ws argument)."""
+    _check(lib().h3_ffn_swiglu_noalloc(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                                       _ptr(xm, BF16, "xm"), _ptr(Wgu, BF16, "Wgu"), _ptr(Wd, BF16, "Wd"),
+                                       _ptr(mod, F32, "mod"), _stream(stream)))
 
 
 def h3_head_unpack(dims, ranges, x, W_vhead, W_ahead, video_shape, audio_shape, hn, v_video, v_audio, stream=None):
