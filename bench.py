@@ -64,6 +64,12 @@ def bytes_per_call(w, L, Lp):
     }
 
 
+# DRAM bytes (read + write) per launch from one ncu capture of the kernel on
+# this workload, valid for the kernel as it was when captured; None once the
+# kernel changes (see profiles/).
+TRAFFIC = {}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason sampling during the timed region."""
 
@@ -248,8 +254,19 @@ def run_ours(args, w):
     fl = flops_per_call(w, L)
     by = bytes_per_call(w, L, Lp)
     tensor_calls = {c: fl[c] / (per_call[c] / 1e3) / 1e12 for c in fl}
-    dominant = max(fl, key=lambda c: per_call[c])
     peak_tf = peaks["bf16_tflops_sustained"]
+    # Kernels: gemm_tc_kernel runs the QKV, out-projection, FFN gate/up and FFN
+    # down launches (the embed/head launches add < 0.4% of its FLOPs and are
+    # not timed separately); attention_tc_kernel is one launch per step.
+    gemm_calls = ("h3_qkv_qknorm_mrope", "h3_gated_residual", "h3_ffn_swiglu")
+    gemm_ms = sum(per_call[c] for c in gemm_calls)
+    gemm_tf = sum(fl[c] for c in gemm_calls) / (gemm_ms / 1e3) / 1e12
+    attn_tf = tensor_calls["h3_attention"]
+    kernels = {"gemm_tc_kernel": {"ms_per_step": round(gemm_ms, 4), "launches_per_step": 4,
+                                  "tflops": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4)},
+               "attention_tc_kernel": {"ms_per_step": round(per_call["h3_attention"], 4), "launches_per_step": 1,
+                                       "tflops": round(attn_tf, 1), "frac": round(attn_tf / peak_tf, 4)}}
+    dominant = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     block_flops = sum(fl.values())
     block_ms = sum(per_call[c] for c in ("h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
                                          "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu"))
@@ -266,10 +283,11 @@ def run_ours(args, w):
                    "l2": "inputs larger than L2: %.0f MB of weights + %.0f MB residual stream read per step" % (
                        sum(t.numel() * 2 for t in W.values()) / 1e6, Lp * w.D * 4 / 1e6)},
         "roofline": {"bound": "tensor", "kernel": dominant,
-                     "achieved": round(tensor_calls[dominant], 1),
-                     "peak": peak_tf, "unit": "TFLOP/s", "frac": round(tensor_calls[dominant] / peak_tf, 4),
-                     "peak_kind": f"bf16 sustained ({peaks['source']})",
-                     "traffic": None},
+                     "achieved": kernels[dominant]["tflops"],
+                     "peak": peak_tf, "unit": "TFLOP/s", "frac": kernels[dominant]["frac"],
+                     "peak_kind": f"bf16 sustained, of measured ({peaks['source']})",
+                     "traffic": TRAFFIC.get((w.name, dominant))},
+        "kernels": kernels,
         "block": {"tflops": round(block_flops / (block_ms / 1e3) / 1e12, 1),
                   "frac_of_bf16_sustained": round(block_flops / (block_ms / 1e3) / 1e12 / peak_tf, 4),
                   "frac_of_bf16_spec_2250": round(block_flops / (block_ms / 1e3) / 1e12 / 2250.0, 4),
@@ -284,6 +302,58 @@ def run_ours(args, w):
     if not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
     return out
+
+
+def run_only(args, w):
+    """One C-ABI call on the workload's shapes, nothing else resident but its
+    operands (for ncu captures of a single kernel)."""
+    import torch
+    from omni_modal_diffusion_b200 import h3
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(4321)
+    rnd = lambda *s, std=1.0, dt=torch.bfloat16: (torch.randn(*s, generator=g, device=dev) * std).to(dt)
+    d = h3.make_dims(w.D, w.H, w.F, rope=w.rope_split)
+    r = h3.h3_make_ranges(w.n_text, w.audio_channels * w.n_audio, w.T_lat * (w.H_lat // 2) * (w.W_lat // 2))
+    Lp = r.L_pad
+    mod = rnd(3, 6, w.D, std=0.1, dt=torch.float32)
+    if args.only == "attention":
+        q, k, v = (rnd(w.H, Lp, 128) for _ in range(3))
+        o = torch.empty(Lp, w.I, dtype=torch.bfloat16, device=dev)
+        fn = lambda: h3.h3_attention(d, r, q, k, v, o)
+    elif args.only == "qkv":
+        xm = rnd(Lp, w.D)
+        Wqkv = rnd(3 * w.I, w.D, std=0.02)
+        qn, kn = rnd(128, std=0.1) + 1, rnd(128, std=0.1) + 1
+        pos = torch.zeros(Lp, 3, device=dev)
+        q, k, v = (torch.empty(w.H, Lp, 128, dtype=torch.bfloat16, device=dev) for _ in range(3))
+        fn = lambda: h3.h3_qkv_qknorm_mrope(d, r, xm, Wqkv, qn, kn, pos, q, k, v)
+    elif args.only == "out":
+        x = rnd(Lp, w.D, dt=torch.float32)
+        o = rnd(Lp, w.I)
+        Wo = rnd(w.D, w.I, std=0.02)
+        fn = lambda: h3.h3_gated_residual(d, r, x, o, Wo, mod, h3.H3_MSA)
+    elif args.only == "ffn":
+        x = rnd(Lp, w.D, dt=torch.float32)
+        xm = rnd(Lp, w.D)
+        Wgu, Wd = rnd(2 * w.F, w.D, std=0.02), rnd(w.D, w.F, std=0.02)
+        ws = torch.empty(Lp, w.F, dtype=torch.bfloat16, device=dev)
+        fn = lambda: h3.h3_ffn_swiglu(d, r, x, xm, Wgu, Wd, mod, ws)
+    else:
+        x = rnd(Lp, w.D, dt=torch.float32)
+        xm = torch.empty(Lp, w.D, dtype=torch.bfloat16, device=dev)
+        fn = lambda: h3.h3_adaln_norm_modulate(d, r, x, mod, h3.H3_MSA, xm)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    print(f"{args.only} on {w.name}: {a.elapsed_time(b) / args.steps:.4f} ms per call", flush=True)
 
 
 def cpu_baseline(w, rows_sample=32):
@@ -349,8 +419,10 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln"],
+                    help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -362,6 +434,9 @@ def main():
         args.warmup = 1            # each oracle step is a ~10-30 s CPU sample
     from omni_modal_diffusion_b200 import synthetic as S
     w = S.WORKLOADS[args.workload]
+    if args.only:
+        run_only(args, w)
+        return
     out = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if out is not None:
         print(json.dumps(out), flush=True)
