@@ -300,7 +300,7 @@ def run_ours(args, w):
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
+        out["cpu_baseline"] = cpu_baseline(w)
     return out
 
 
@@ -356,11 +356,19 @@ def run_only(args, w):
     print(f"{args.only} on {w.name}: {a.elapsed_time(b) / args.steps:.4f} ms per call", flush=True)
 
 
-def cpu_baseline(w, rows_sample=32):
+def block_flops(w, L):
+    """Algorithmic FLOPs of one block over L valid tokens."""
+    return 2.0 * L * (w.D * 3 * w.I + w.I * w.D + 2 * w.D * w.F + w.F * w.D) + 4.0 * L * L * w.I
+
+
+def cpu_baseline(w, frames=2):
     """The float64 oracle on the host cores, on a bounded sample of the same
-    workload: K and V of every token (all of them feed attention) plus the
-    full block for `rows_sample` query rows; the per-row part is scaled to all
-    L rows (the block's cost is exactly K/V for all tokens + per-row work)."""
+    workload: the whole block (packing, projections, LN+modulate, QKV,
+    RMSNorm, RoPE, attention, gated out-projection, SwiGLU FFN) on the same
+    text and audio with the video cut to `frames` latent frames, timed in
+    full, then scaled to the workload's length by the block's algorithmic
+    FLOPs (the oracle is matmul-bound)."""
+    import dataclasses
     from oracle import h3_oracle as O
     from omni_modal_diffusion_b200 import synthetic as S
     try:
@@ -368,27 +376,24 @@ def cpu_baseline(w, rows_sample=32):
         threads = max(info.get("num_threads", 0) for info in threadpoolctl.threadpool_info()) or os.cpu_count()
     except Exception:  # pragma: no cover
         threads = os.cpu_count()
-    inp = S.make_inputs(w)
-    t_g, i_g, j_g = O.token_grid(w.T_lat, w.H_lat, w.W_lat)
-    r = O.pack_ranges(w.n_text, w.audio_channels * w.n_audio, t_g * i_g * j_g)
-    pos = O.positions(r, t_g, i_g, j_g, w.audio_channels, w.n_audio)
+    ws = dataclasses.replace(w, T_lat=min(frames, w.T_lat))
+    inp = S.make_inputs(ws)
+    t_g, i_g, j_g = O.token_grid(ws.T_lat, ws.H_lat, ws.W_lat)
+    r = O.pack_ranges(ws.n_text, ws.audio_channels * ws.n_audio, t_g * i_g * j_g)
+    pos = O.positions(r, t_g, i_g, j_g, ws.audio_channels, ws.n_audio)
+    t0 = time.perf_counter()
     x = O.embed(inp["text"], inp["video"], inp["audio"], inp["W_text"], inp["W_vid"], inp["W_aud"], r)
-    L = r["L"]
-    rows = S.random_rows(L, rows_sample, seed=99)
-    t0 = time.perf_counter()
-    O.block_forward_rows(x, inp["mod"], r, pos, rows[:1], inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"],
-                         inp["Wgu"], inp["Wd"], w.H)
-    t_kv = time.perf_counter() - t0       # K/V for all tokens + 1 row
-    t0 = time.perf_counter()
-    O.block_forward_rows(x, inp["mod"], r, pos, rows, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"],
-                         inp["Wgu"], inp["Wd"], w.H)
-    t_all = time.perf_counter() - t0
-    per_row = max(t_all - t_kv, 1e-9) / (len(rows) - 1)
-    t_block = (t_kv - per_row) + per_row * L
-    return {"value": round(L / t_block, 3), "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"float64 oracle block on {w.name}: K/V of all {L} tokens + {len(rows)} sampled query rows "
-                      f"({t_kv + t_all:.1f} s measured), per-row time scaled to {L} rows",
-            "seconds_per_block_extrapolated": round(t_block, 2)}
+    O.block_forward(x, inp["mod"], r, pos, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"], inp["Wgu"],
+                    inp["Wd"], ws.H)
+    t_s = time.perf_counter() - t0
+    Ls = r["L"]
+    L = w.n_text + w.audio_channels * w.n_audio + w.T_lat * (w.H_lat // 2) * (w.W_lat // 2)
+    t_full = t_s * block_flops(w, L) / block_flops(w, Ls)
+    return {"value": round(L / t_full, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"float64 oracle block on {w.name} cut to {ws.T_lat} latent frames ({Ls} packed tokens, "
+                      f"{t_s:.1f} s measured), scaled to {L} tokens by algorithmic FLOPs "
+                      f"({block_flops(w, L) / block_flops(w, Ls):.2f}x)",
+            "seconds_per_block_extrapolated": round(t_full, 2)}
 
 
 def run_reference(args, w):
@@ -400,7 +405,7 @@ def run_reference(args, w):
     base = None
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        cb = cpu_baseline(w, args.cpu_rows)
+        cb = cpu_baseline(w)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             vals.append(cb["value"])
@@ -426,7 +431,6 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=24)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

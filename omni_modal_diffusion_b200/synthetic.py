@@ -67,12 +67,15 @@ WORKLOADS = {
 def bf16_round(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); float32 out."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) << 16
-    out = r.astype(np.uint32).view(np.float32)
-    # keep NaN as NaN (not produced by these generators, kept for safety)
-    return np.where(np.isnan(a), a, out)
+    u = a.view(np.uint32)
+    r = u + np.uint32(0x7FFF)                 # new array: the input is not modified
+    r += (u >> np.uint32(16)) & np.uint32(1)
+    r &= np.uint32(0xFFFF0000)
+    out = r.view(np.float32)
+    nan = np.isnan(a)
+    if nan.any():
+        out[nan] = a[nan]
+    return out
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -82,7 +85,12 @@ def bf16_bits(a: np.ndarray) -> np.ndarray:
 
 
 def _normal(rng, shape, std=1.0, mean=0.0):
-    return (rng.standard_normal(size=shape, dtype=np.float32) * np.float32(std) + np.float32(mean))
+    a = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    if mean != 0.0:
+        a += np.float32(mean)
+    return a
 
 
 def make_inputs(w: Workload, seed: int | None = None, weights: bool = True) -> dict:

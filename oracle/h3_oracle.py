@@ -330,21 +330,26 @@ def block_forward(x, mod, ranges, pos, Wqkv, qn_w, kn_w, Wo, Wgu, Wd, n_heads,
 def block_forward_rows(x, mod, ranges, pos, rows, Wqkv, qn_w, kn_w, Wo, Wgu, Wd, n_heads,
                        head_dim=128, split=(32, 48, 48)):
     """`block_forward` evaluated only at the given output rows.  K and V are
-    computed for every token (attention reads all of them); everything
-    row-local is computed for the sampled rows only.  Same formulas."""
+    computed for every token (attention reads all of them), one head at a
+    time so that memory stays at one head's K/V; everything row-local is
+    computed for the sampled rows only.  Same formulas as `block_forward`."""
     x = np.asarray(x, np.float64)
-    L = x.shape[0]
+    rows = np.asarray(rows)
     I = n_heads * head_dim
     xm_all = adaln_modulate(x, mod, ranges, MSA)
-    kv = linear(xm_all, Wqkv[I:])
-    k = rope(rmsnorm(kv[:, :I].reshape(L, n_heads, head_dim), kn_w), pos, split)
-    v = kv[:, I:].reshape(L, n_heads, head_dim)
-    q = linear(xm_all[rows], Wqkv[:I]).reshape(len(rows), n_heads, head_dim)
-    q = rope(rmsnorm(q, qn_w), pos[rows], split)
-    o = attention_rows(q, k, v)
+    o = np.empty((len(rows), n_heads, head_dim), dtype=np.float64)
+    for h in range(n_heads):
+        cols = slice(h * head_dim, (h + 1) * head_dim)
+        wq = Wqkv[0 * I:1 * I][cols]
+        wk = Wqkv[1 * I:2 * I][cols]
+        wv = Wqkv[2 * I:3 * I][cols]
+        k = rope(rmsnorm(linear(xm_all, wk)[:, None, :], kn_w), pos, split)
+        v = linear(xm_all, wv)[:, None, :]
+        q = rope(rmsnorm(linear(xm_all[rows], wq)[:, None, :], qn_w), pos[rows], split)
+        o[:, h, :] = attention_rows(q, k, v)
+    o = o.reshape(len(rows), I)
     x1 = gated_residual(x[rows], o, Wo, mod, ranges, rows)
-    sub = {"start": ranges["start"], "count": ranges["count"], "L": ranges["L"]}
-    m = modality_of_rows(sub)[rows]
+    m = modality_of_rows(ranges)[rows]
     modv = np.asarray(mod, np.float64)
     xm2 = layernorm(x1) * (1.0 + modv[m, 3 * MLP + SCALE]) + modv[m, 3 * MLP + SHIFT]
     x2 = ffn_swiglu(x1, xm2, Wgu, Wd, mod, ranges, rows)
