@@ -206,6 +206,13 @@ int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x,
  * [shouss] §5, §6).  lat, vel: fp32 device arrays of n elements. */
 int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream);
 
+/* Diagnostic: y[i] = 2^x[i] computed the way h3_attention computes a quarter
+ * of its softmax exponentials on full key tiles, on the FMA pipe instead of
+ * the MUFU unit: x clamped to >= -125, x = j + f with j = rint(x), 2^f from a
+ * cubic (max relative error 7.5e-5 for x in [-125, 64]), 2^j added to the
+ * exponent.  x, y: fp32 device arrays of n elements. */
+int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream);
+
 /* Synchronise `stream`, then report (and clear) the device error word that
  * bounded device-side waits set when they give up.  *code_out = 0 when no
  * wait failed.  Returns H3_ERR_TIMEOUT if one did, H3_ERR_CUDA on a CUDA

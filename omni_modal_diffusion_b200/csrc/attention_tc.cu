@@ -36,6 +36,20 @@ constexpr int SMEM_BAR = SMEM_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// Tuning knobs (compile time): one pair in POLY_EVERY pairs of a full key
+// tile takes its exponentials on the FMA pipe (0 = none); SPLIT_P releases
+// P to the PV MMA in two halves instead of one.  Measured on B200 at 7,904
+// and 32,160 tokens: POLY_EVERY 0 / 8 / 4 / 2 -> 1.64 / 1.65 / 1.66-1.76 /
+// 1.70-1.78 ms and SPLIT_P 1 is 4-8% slower, because each softmax thread's
+// instruction latency, not MUFU throughput, bounds a phase in this layout.
+#ifndef H3_ATTN_POLY_EVERY
+#define H3_ATTN_POLY_EVERY 0
+#endif
+#ifndef H3_ATTN_SPLIT_P
+#define H3_ATTN_SPLIT_P 0
+#endif
+constexpr int POLY_EVERY = H3_ATTN_POLY_EVERY;
+constexpr bool SPLIT_P = H3_ATTN_SPLIT_P != 0;
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -49,13 +63,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sV = smem + SMEM_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2] per stage
-  uint64_t* v_full = bars + 3;    // [2] per stage
-  uint64_t* kv_empty = bars + 5;  // [2] per stage
-  uint64_t* s_full = bars + 7;    // [2] per query tile
-  uint64_t* p_full = bars + 9;    // [2] per query tile
+  uint64_t* k_full = bars + 1;    // [2] per K stage
+  uint64_t* v_full = bars + 3;    // [2] per V stage
+  uint64_t* k_empty = bars + 5;   // [2] per K stage: freed after the tile's last S MMA
+  uint64_t* v_empty = bars + 7;   // [2] per V stage: freed after the tile's last PV MMA
+  uint64_t* s_full = bars + 9;    // [2] per query tile
   uint64_t* o_final = bars + 11;  // [2] per query tile
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* p_full = bars + 13;   // [2 tiles][2 halves of the key tile]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -70,9 +85,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[2 * s], 4);
+      mbar_init(&p_full[2 * s + 1], 4);
       mbar_init(&o_final[s], 1);
     }
     fence_mbar_init();
@@ -98,12 +115,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_load_2d(sQ + TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, row0 + qt1 * TILE);
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
-        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1)) break;
         uint8_t* dk = sK + st * TILE_BYTES;
         uint8_t* dv = sV + st * TILE_BYTES;
+        if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
         tma_load_2d(dk, &tmK, &k_full[st], 0, row0 + j * TILE);
         tma_load_2d(dk + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
+        if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
         tma_load_2d(dv, &tmV, &v_full[st], 0, row0 + j * TILE);
         tma_load_2d(dv + HALF_BYTES, &tmV, &v_full[st], 64, row0 + j * TILE);
@@ -126,33 +144,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         umma_commit(&s_full[t]);
       };
-      // O_t += P_t V_j, P_t (bf16, packed) read from TMEM where S_t was
-      auto issue_pv = [&](int t, int j) {
+      // O_t += P_t V_j for keys [64 hf, 64 hf + 64), P_t (bf16, packed)
+      // read from TMEM where S_t was
+      auto issue_pv_half = [&](int t, int j, int hf) {
         const uint32_t v_addr = smem_u32(sV + (j & 1) * TILE_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = hf * 4 + k4;
           const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024);
           umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, bd, idesc_o, (j | kk) != 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0) && mbar_wait(&k_full[0], 0);
+      bool ok = mbar_wait_spin(q_full, 0) && mbar_wait_spin(&k_full[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
+        umma_commit(&k_empty[0]);
       }
       for (int j = 0; j < nkv && ok; ++j) {
         const bool more = j + 1 < nkv;
-        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1)) break;
-        if (more && !mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) break;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!mbar_wait(&p_full[t], j & 1)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(t, j);
-          if (more) issue_s(t, j + 1);
-          else umma_commit(&o_final[t]);
+          for (int hf = 0; hf < 2; ++hf) {
+            if (SPLIT_P || hf == 0) {
+              if (!mbar_wait_spin(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
+              if (t == 0 && hf == 0 && !mbar_wait_spin(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_pv_half(t, j, hf);
+          }
+          if (!ok) break;
+          if (more) {
+            if (t == 0) {
+              if (!mbar_wait_spin(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_s(t, j + 1);
+            if (t == 1) umma_commit(&k_empty[(j + 1) & 1]);
+          } else {
+            umma_commit(&o_final[t]);
+          }
         }
-        umma_commit(&kv_empty[j & 1]);
+        umma_commit(&v_empty[j & 1]);
       }
     }
   } else {
@@ -174,10 +207,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_wait_ld();
 
       const int valid = L - j * TILE;  // keys [0, valid) of this tile are real
+      const bool full = valid >= TILE;
       float mx = -INFINITY;
-      if (valid >= TILE) {
+      if (full) {
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 128; c += 8) {
+          m4[0] = max3f(m4[0], s[c], s[c + 1]);
+          m4[1] = max3f(m4[1], s[c + 2], s[c + 3]);
+          m4[2] = max3f(m4[2], s[c + 4], s[c + 5]);
+          m4[3] = max3f(m4[3], s[c + 6], s[c + 7]);
+        }
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       } else {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
@@ -201,22 +242,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_st32(tO + c * 32, reinterpret_cast<const uint32_t*>(o));
         }
       }
-      float rs = 0.f;
-      uint32_t pk[64];
+      // p = 2^(s * scale_log2 - m_ref); on full tiles some exponentials run
+      // on the FMA pipe (exp2_poly2) to relieve the MUFU unit; masked tiles
+      // use ex2 only so that masked keys give exactly 0.
+      const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+      // P for keys [64 hf, 64 hf + 64) goes to TMEM columns [32 hf, 32 hf + 32)
+      // (it only overwrites S columns already in registers)
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(s[c], scale_log2, -m_ref));
-        const float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, -m_ref));
-        rs += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const int cc = hf * 64 + c;
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(s[cc], s[cc + 1]), sc2, nm2), x0, x1);
+          if (POLY_EVERY > 0 && full && ((c / 2) % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
+            exp2_poly2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_pack(p0, p1));
+          pk[c / 2] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + hf * 32, pk);
+        if (SPLIT_P || hf == 1) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[2 * t + (SPLIT_P ? hf : 0)]);
+        }
       }
-      l_sum = fmaf(l_sum, alpha, rs);
-      tmem_st32(tS, pk);
-      tmem_st32(tS + 32, pk + 32);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t]);
+      float a0, a1, a2, a3;
+      f2_unpack(acc[0], a0, a1);
+      f2_unpack(acc[1], a2, a3);
+      l_sum = fmaf(l_sum, alpha, (a0 + a1) + (a2 + a3));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
     const int qt = t == 0 ? qt0 : qt1;

@@ -169,6 +169,24 @@ __global__ void euler_kernel(float* __restrict__ lat, const float* __restrict__ 
     lat[i] = fmaf(dsigma, vel[i], lat[i]);
 }
 
+// The attention softmax's FMA-pipe exponential on an array (for checking it
+// against its error bound).
+__global__ void exp2_fma_pipe_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long pairs = n / 2;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < pairs;
+       i += (long long)gridDim.x * blockDim.x) {
+    float y0, y1;
+    exp2_poly2(x[2 * i], x[2 * i + 1], y0, y1);
+    y[2 * i] = y0;
+    y[2 * i + 1] = y1;
+  }
+  if (n & 1 && blockIdx.x == 0 && threadIdx.x == 0) {
+    float y0, y1;
+    exp2_poly2(x[n - 1], x[n - 1], y0, y1);
+    y[n - 1] = y0;
+  }
+}
+
 }  // namespace ew_detail
 using namespace ew_detail;
 
@@ -208,6 +226,15 @@ cudaError_t launch_ln_modulate(const float* x, const float* mod, int branch, con
     rg.count[m] = rcount[m];
   }
   ln_modulate_kernel<<<L_pad, LN_THREADS, 0, stream>>>(x, mod, branch, rg, L, D, eps, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_exp2_fma_pipe(const float* x, float* y, long long n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  long long blocks = (n / 2 + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 148LL * 8) blocks = 148LL * 8;
+  exp2_fma_pipe_kernel<<<(int)blocks, 256, 0, stream>>>(x, y, n);
   return cudaGetLastError();
 }
 

@@ -398,6 +398,16 @@ int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float si
   return ok();
 }
 
+int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return fail(H3_ERR_SHAPE, "h3_exp2_fma_pipe: n < 0");
+  if (n == 0) return ok();
+  H3_REQUIRE_PTR(x);
+  H3_REQUIRE_PTR(y);
+  cudaError_t e = launch_exp2_fma_pipe(x, y, (long long)n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_exp2_fma_pipe");
+  return ok();
+}
+
 int h3_device_status(void* stream, int* code_out) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: synchronize");

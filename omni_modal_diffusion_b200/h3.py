@@ -24,7 +24,7 @@ EXPORTS = (
     "h3_last_error", "h3_version", "h3_make_ranges", "h3_sigma_schedule", "h3_embed_pack",
     "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention", "h3_gated_residual",
     "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
-    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc",
+    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_exp2_fma_pipe",
 )
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
 
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "h3_ffn_swiglu_noalloc": (ci, [pd, pr, vp, vp, vp, vp, vp, vp]),
             "h3_head_unpack": (ci, [pd, pr, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]),
             "h3_euler_step": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp]),
+            "h3_exp2_fma_pipe": (ci, [vp, vp, ctypes.c_int64, vp]),
             "h3_device_status": (ci, [vp, ctypes.POINTER(ci)]),
             "h3_set_wait_limit_ns": (ci, [ctypes.c_uint64]),
         }
@@ -193,6 +194,10 @@ def h3_euler_step(lat, vel, sigma: float, sigma_next: float, stream=None):
         raise ValueError("lat and vel sizes differ")
     _check(lib().h3_euler_step(_ptr(lat, F32, "lat"), _ptr(vel, F32, "vel"), lat.numel(), sigma, sigma_next,
                                _stream(stream)))
+
+
+def h3_exp2_fma_pipe(x, y, stream=None):
+    _check(lib().h3_exp2_fma_pipe(_ptr(x, F32, "x"), _ptr(y, F32, "y"), x.numel(), _stream(stream)))
 
 
 def h3_device_status(stream=None) -> int:

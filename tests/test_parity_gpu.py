@@ -385,3 +385,21 @@ def test_full_length_qkv_sampled_rows():
 
 def test_device_status_clean_after_work():
     assert h3.h3_device_status() == 0
+
+
+def test_exp2_fma_pipe_error_bound():
+    """The softmax's FMA-pipe exponential stays within its stated 7.5e-5
+    relative error of 2^x over the range the softmax feeds it (x <= 8 after
+    the lazy max; down to the -125 clamp), and matches the clamp below."""
+    x = np.concatenate([np.linspace(-125.0, 64.0, 2_000_001), np.arange(-125, 64, dtype=np.float64) + 0.5,
+                        np.arange(-125, 65, dtype=np.float64)]).astype(np.float32)
+    y = torch.empty(len(x), device=DEV)
+    h3.h3_exp2_fma_pipe(_f32(x), y)
+    got = to_np(y)
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(got / ref - 1.0)
+    assert rel.max() <= 7.6e-5, rel.max()
+    z = torch.empty(3, device=DEV)
+    h3.h3_exp2_fma_pipe(_f32(np.array([-200.0, -1e30, -125.0], np.float32)), z)
+    zz = to_np(z)
+    assert np.allclose(zz, 2.0 ** -125, rtol=1e-4)
