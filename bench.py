@@ -304,6 +304,62 @@ def run_ours(args, w):
     return out
 
 
+def run_sampler(args, w):
+    """The layered flow sampler: args.layers blocks per denoise step, timed
+    over args.steps denoise steps (after args.warmup untimed ones)."""
+    import torch
+    from omni_modal_diffusion_b200 import h3
+    from omni_modal_diffusion_b200.pipeline import H3Sampler
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(99 + w.index)
+    rnd = lambda *s, std=1.0, dt=torch.bfloat16: (torch.randn(*s, generator=g, device=dev) * std).to(dt)
+    io = {"W_text": rnd(w.D, w.D_text, std=0.02), "W_vid": rnd(w.D, 4 * w.C_lat, std=0.02),
+          "W_aud": rnd(w.D, w.C_audio, std=0.02), "W_vhead": rnd(4 * w.C_lat, w.D, std=0.02),
+          "W_ahead": rnd(w.C_audio, w.D, std=0.02)}
+    blocks = [{"Wqkv": rnd(3 * w.I, w.D, std=0.02), "qn_w": rnd(128, std=0.1) + 1, "kn_w": rnd(128, std=0.1) + 1,
+               "Wo": rnd(w.D, w.I, std=0.02), "Wgu": rnd(2 * w.F, w.D, std=0.02), "Wd": rnd(w.D, w.F, std=0.02)}
+              for _ in range(args.layers)]
+    smp = H3Sampler(w, io, blocks, device=dev)
+    L = smp.st.ranges.L
+    n_total = args.warmup + args.steps
+    text = rnd(w.n_text, w.D_text)
+    lv = rnd(w.T_lat, w.H_lat, w.W_lat, w.C_lat, dt=torch.float32)
+    la = rnd(w.audio_channels, w.n_audio, w.C_audio, dt=torch.float32)
+    lv_bf, la_bf = lv.to(torch.bfloat16), la.to(torch.bfloat16)
+    mod_all = rnd(n_total, args.layers, 3, 6, w.D, std=0.1, dt=torch.float32)
+    sv = h3.h3_sigma_schedule(n_total, 12.0)
+    sa = h3.h3_sigma_schedule(n_total, 3.0)
+    stream = torch.cuda.current_stream(dev)
+    for s in range(args.warmup):
+        smp.step(s, text, lv, la, lv_bf, la_bf, mod_all, sv, sa)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(args.warmup, n_total):
+        smp.step(s, text, lv, la, lv_bf, la_bf, mod_all, sv, sa)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    assert h3.h3_device_status() == 0
+    ms = a.elapsed_time(b) / args.steps
+    fl = block_flops(w, L) * args.layers
+    return {"metric": "end-to-end denoise steps/s (layered flow sampler, bf16, 1xB200)",
+            "value": round(1e3 / ms, 4), "unit": "denoise steps/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init bf16 weights, N(0,1) latents)",
+            "config": {"workload": w.name, "packed_tokens": L, "layers": args.layers,
+                       "weights_gb": round(sum(t.numel() * 2 for b_ in blocks for t in b_.values()) / 1e9, 1)},
+            "tokens_per_s_per_block": round(L * args.layers / (ms / 1e3), 1),
+            "tflops": round(fl / (ms / 1e3) / 1e12, 1), "frac_of_bf16_sustained": round(
+                fl / (ms / 1e3) / 1e12 / _peaks()["bf16_tflops_sustained"], 4),
+            "gpu_launches": smp.launches_per_step() * args.steps, "clocks": clocks}
+
+
 def run_only(args, w):
     """One C-ABI call on the workload's shapes, nothing else resident but its
     operands (for ncu captures of a single kernel)."""
@@ -424,22 +480,32 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 100; sampler: 8)")
+    ap.add_argument("--warmup", type=int, default=None, help="untimed steps (default 10; sampler: 3)")
+    ap.add_argument("--sampler", action="store_true",
+                    help="time the layered flow sampler (denoise steps/s) instead of the single-block step")
+    ap.add_argument("--layers", type=int, default=50)
     ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None, help=f"default {DEFAULT_WORKLOAD}; sampler: 768x1344_5s")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 8 if args.sampler else 100
+    if args.warmup is None:
+        args.warmup = 3 if args.sampler else 10
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference" and args.warmup > 1:
         args.warmup = 1            # each oracle step is a ~10-30 s CPU sample
     from omni_modal_diffusion_b200 import synthetic as S
-    w = S.WORKLOADS[args.workload]
+    w = S.WORKLOADS[args.workload or ("768x1344_5s" if args.sampler else DEFAULT_WORKLOAD)]
     if args.only:
         run_only(args, w)
+        return
+    if args.sampler:
+        print(json.dumps(run_sampler(args, w)), flush=True)
         return
     out = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
     if out is not None:

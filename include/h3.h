@@ -213,6 +213,40 @@ int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float si
  * exponent.  x, y: fp32 device arrays of n elements. */
 int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream);
 
+/* Block weights and scratch buffers for h3_block_forward (all device
+ * pointers, layouts as in the individual calls). */
+typedef struct h3_block_weights {
+  const h3_bf16* Wqkv; /* [3I][D] */
+  const h3_bf16* qn_w; /* [128] */
+  const h3_bf16* kn_w; /* [128] */
+  const h3_bf16* Wo;   /* [D][I] */
+  const h3_bf16* Wgu;  /* [2F][D], gate rows then up rows */
+  const h3_bf16* Wd;   /* [D][F] */
+} h3_block_weights;
+
+typedef struct h3_block_buffers {
+  h3_bf16* xm;         /* [L_pad][D] */
+  h3_bf16* q;          /* [H][L_pad][128] */
+  h3_bf16* k;          /* [H][L_pad][128] */
+  h3_bf16* v;          /* [H][L_pad][128] */
+  h3_bf16* o;          /* [L_pad][I] */
+  h3_bf16* ws;         /* h3_ffn_workspace_bytes() */
+} h3_block_buffers;
+
+/* One whole block on x in place: h3_adaln_norm_modulate (MSA),
+ * h3_qkv_qknorm_mrope, h3_attention, h3_gated_residual, h3_adaln_norm_modulate
+ * (MLP), h3_ffn_swiglu, in the order of [shouss] §3 (norm + modality
+ * shift/scale -> shared attention + gate + residual -> norm + shift/scale ->
+ * shared gated FFN + gate + residual).  Same arguments and errors as those
+ * calls; nothing is launched if any argument is invalid. */
+int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod, const float* pos,
+                     const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream);
+
+/* A11 for a sampler loop: h3_euler_step, and also writes the updated latent
+ * rounded to bf16 into lat_bf16 (the transformer input of the next step). */
+int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, h3_bf16* lat_bf16,
+                       void* stream);
+
 /* Synchronise `stream`, then report (and clear) the device error word that
  * bounded device-side waits set when they give up.  *code_out = 0 when no
  * wait failed.  Returns H3_ERR_TIMEOUT if one did, H3_ERR_CUDA on a CUDA

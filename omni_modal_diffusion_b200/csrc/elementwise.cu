@@ -169,6 +169,30 @@ __global__ void euler_kernel(float* __restrict__ lat, const float* __restrict__ 
     lat[i] = fmaf(dsigma, vel[i], lat[i]);
 }
 
+// Euler update that also writes the bf16 copy the next step's packing reads.
+__global__ void euler_bf16_kernel(float* __restrict__ lat, const float* __restrict__ vel, long long n, float dsigma,
+                                  bf16* __restrict__ out) {
+  const long long nv = n / 4;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  float4* l4 = reinterpret_cast<float4*>(lat);
+  const float4* v4 = reinterpret_cast<const float4*>(vel);
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nv; i += stride) {
+    float4 a = l4[i];
+    const float4 b = __ldcs(v4 + i);
+    a.x = fmaf(dsigma, b.x, a.x);
+    a.y = fmaf(dsigma, b.y, a.y);
+    a.z = fmaf(dsigma, b.z, a.z);
+    a.w = fmaf(dsigma, b.w, a.w);
+    l4[i] = a;
+    *reinterpret_cast<uint2*>(out + 4 * i) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+  for (long long i = nv * 4 + blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float a = fmaf(dsigma, vel[i], lat[i]);
+    lat[i] = a;
+    out[i] = __float2bfloat16_rn(a);
+  }
+}
+
 // The attention softmax's FMA-pipe exponential on an array (for checking it
 // against its error bound).
 __global__ void exp2_fma_pipe_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
@@ -235,6 +259,16 @@ cudaError_t launch_exp2_fma_pipe(const float* x, float* y, long long n, cudaStre
   if (blocks < 1) blocks = 1;
   if (blocks > 148LL * 8) blocks = 148LL * 8;
   exp2_fma_pipe_kernel<<<(int)blocks, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_euler_bf16(float* lat, const float* vel, long long n, float dsigma, bf16* out,
+                              cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  long long blocks = (n / 4 + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 148LL * 8) blocks = 148LL * 8;
+  euler_bf16_kernel<<<(int)blocks, 256, 0, stream>>>(lat, vel, n, dsigma, out);
   return cudaGetLastError();
 }
 

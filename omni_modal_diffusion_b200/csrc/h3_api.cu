@@ -398,6 +398,52 @@ int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float si
   return ok();
 }
 
+int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, h3_bf16* lat_bf16,
+                       void* stream) {
+  if (n < 0) return fail(H3_ERR_SHAPE, "h3_euler_step_bf16: n < 0");
+  if (n == 0) return ok();
+  H3_REQUIRE_PTR(lat);
+  H3_REQUIRE_PTR(vel);
+  H3_REQUIRE_PTR(lat_bf16);
+  cudaError_t e = launch_euler_bf16(lat, vel, (long long)n, sigma_next - sigma, reinterpret_cast<bf16*>(lat_bf16),
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_euler_step_bf16");
+  return ok();
+}
+
+int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod, const float* pos,
+                     const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  if (!w) return fail(H3_ERR_NULL, "%s: weights is NULL", __func__);
+  if (!buf) return fail(H3_ERR_NULL, "%s: buffers is NULL", __func__);
+  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
+    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  H3_REQUIRE_PTR(x);
+  H3_REQUIRE_PTR(mod);
+  H3_REQUIRE_PTR(pos);
+  H3_REQUIRE_PTR(w->Wqkv);
+  H3_REQUIRE_PTR(w->qn_w);
+  H3_REQUIRE_PTR(w->kn_w);
+  H3_REQUIRE_PTR(w->Wo);
+  H3_REQUIRE_PTR(w->Wgu);
+  H3_REQUIRE_PTR(w->Wd);
+  H3_REQUIRE_PTR(buf->xm);
+  H3_REQUIRE_PTR(buf->q);
+  H3_REQUIRE_PTR(buf->k);
+  H3_REQUIRE_PTR(buf->v);
+  H3_REQUIRE_PTR(buf->o);
+  H3_REQUIRE_PTR(buf->ws);
+  H3_CHECK(h3_adaln_norm_modulate(dims, ranges, x, mod, H3_MSA, buf->xm, stream));
+  H3_CHECK(h3_qkv_qknorm_mrope(dims, ranges, buf->xm, w->Wqkv, w->qn_w, w->kn_w, pos, flags, buf->q, buf->k, buf->v,
+                               stream));
+  H3_CHECK(h3_attention(dims, ranges, buf->q, buf->k, buf->v, w->qn_w, w->kn_w, pos, flags, buf->o, stream));
+  H3_CHECK(h3_gated_residual(dims, ranges, x, buf->o, w->Wo, mod, H3_MSA, stream));
+  H3_CHECK(h3_adaln_norm_modulate(dims, ranges, x, mod, H3_MLP, buf->xm, stream));
+  H3_CHECK(h3_ffn_swiglu(dims, ranges, x, buf->xm, w->Wgu, w->Wd, mod, buf->ws, stream));
+  return ok();
+}
+
 int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream) {
   if (n < 0) return fail(H3_ERR_SHAPE, "h3_exp2_fma_pipe: n < 0");
   if (n == 0) return ok();

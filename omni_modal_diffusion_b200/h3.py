@@ -24,7 +24,8 @@ EXPORTS = (
     "h3_last_error", "h3_version", "h3_make_ranges", "h3_sigma_schedule", "h3_embed_pack",
     "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention", "h3_gated_residual",
     "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
-    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_exp2_fma_pipe",
+    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_exp2_fma_pipe", "h3_block_forward",
+    "h3_euler_step_bf16",
 )
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
 
@@ -46,6 +47,14 @@ class Ranges(ctypes.Structure):
 
     def as_dict(self) -> dict:
         return {"start": list(self.start), "count": list(self.count), "L": self.L, "L_pad": self.L_pad}
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("Wqkv", "qn_w", "kn_w", "Wo", "Wgu", "Wd")]
+
+
+class BlockBuffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("xm", "q", "k", "v", "o", "ws")]
 
 
 _lib = None
@@ -76,6 +85,9 @@ def lib() -> ctypes.CDLL:
             "h3_head_unpack": (ci, [pd, pr, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]),
             "h3_euler_step": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp]),
             "h3_exp2_fma_pipe": (ci, [vp, vp, ctypes.c_int64, vp]),
+            "h3_euler_step_bf16": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp, vp]),
+            "h3_block_forward": (ci, [pd, pr, vp, vp, vp, ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockBuffers),
+                                      ci, vp]),
             "h3_device_status": (ci, [vp, ctypes.POINTER(ci)]),
             "h3_set_wait_limit_ns": (ci, [ctypes.c_uint64]),
         }
@@ -194,6 +206,29 @@ def h3_euler_step(lat, vel, sigma: float, sigma_next: float, stream=None):
         raise ValueError("lat and vel sizes differ")
     _check(lib().h3_euler_step(_ptr(lat, F32, "lat"), _ptr(vel, F32, "vel"), lat.numel(), sigma, sigma_next,
                                _stream(stream)))
+
+
+def block_weights(W: dict) -> BlockWeights:
+    """Pointer struct of one block's weights (dict of bf16 CUDA tensors)."""
+    return BlockWeights(*(_ptr(W[n], BF16, n) for n in ("Wqkv", "qn_w", "kn_w", "Wo", "Wgu", "Wd")))
+
+
+def block_buffers(xm, q, k, v, o, ws) -> BlockBuffers:
+    return BlockBuffers(*(_ptr(t, BF16, n) for n, t in zip(("xm", "q", "k", "v", "o", "ws"), (xm, q, k, v, o, ws))))
+
+
+def h3_block_forward(dims, ranges, x, mod, pos, weights: BlockWeights, buffers: BlockBuffers,
+                     flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_block_forward(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"), _ptr(mod, F32, "mod"),
+                                  _ptr(pos, F32, "pos"), ctypes.byref(weights), ctypes.byref(buffers), flags,
+                                  _stream(stream)))
+
+
+def h3_euler_step_bf16(lat, vel, sigma: float, sigma_next: float, lat_bf16, stream=None):
+    if lat.numel() != vel.numel() or lat.numel() != lat_bf16.numel():
+        raise ValueError("lat, vel and lat_bf16 sizes differ")
+    _check(lib().h3_euler_step_bf16(_ptr(lat, F32, "lat"), _ptr(vel, F32, "vel"), lat.numel(), sigma, sigma_next,
+                                    _ptr(lat_bf16, BF16, "lat_bf16"), _stream(stream)))
 
 
 def h3_exp2_fma_pipe(x, y, stream=None):

@@ -51,7 +51,11 @@ class H3BlockStep:
             self.load_weights(weights)
 
     def load_weights(self, weights: dict):
+        """Upload the weights present in `weights` (block weights are optional:
+        the layered sampler keeps them per block)."""
         for k in self.WEIGHTS:
+            if k not in weights:
+                continue
             v = weights[k]
             self.W[k] = v if isinstance(v, torch.Tensor) else to_dev_bf16(v, self.device)
 
@@ -98,3 +102,49 @@ class H3BlockStep:
         block = 1 + 1 + 1 + 1 + 1 + 2
         head = 1 + (1 if r.count[2] > 0 else 0) + (1 if r.count[1] > 0 else 0)
         return embed + block + head + 2
+
+
+class H3Sampler:
+    """The 50-block, N-step flow sampler on one GPU ("MiniMax-H3: native joint
+    audio-video generation" §6: separately shifted video / audio schedules,
+    Euler update of the generation targets only; text is a fixed condition).
+
+    Per denoise step: pack + project the bf16 latents, n_layers blocks
+    (h3_block_forward, modulation [step][layer][3][6][D]), head, then one
+    Euler step per modality that also writes the bf16 latent for the next
+    step.  Orchestration only: every step runs in the library's kernels."""
+
+    def __init__(self, w: Workload, io_weights: dict, block_weights: list, device="cuda",
+                 shift_video: float = 12.0, shift_audio: float = 3.0):
+        self.st = H3BlockStep(w, device=device, weights=io_weights)
+        self.block_tensors = block_weights            # keep the tensors alive
+        self.blocks = [h3.block_weights(Wb) for Wb in block_weights]
+        st = self.st
+        self.bufs = h3.block_buffers(st.xm, st.q, st.k, st.v, st.o, st.ws)
+        self.shifts = (shift_video, shift_audio)
+
+    @property
+    def n_layers(self) -> int:
+        return len(self.blocks)
+
+    def step(self, s, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, sv, sa, stream=None):
+        st = self.st
+        st.embed(text, video_bf16, audio_bf16, stream)
+        for b in range(self.n_layers):
+            h3.h3_block_forward(st.dims, st.ranges, st.x, mod_all[s, b], st.pos, self.blocks[b], self.bufs,
+                                stream=stream)
+        st.head(stream)
+        h3.h3_euler_step_bf16(lat_video, st.v_video, sv[s], sv[s + 1], video_bf16, stream=stream)
+        h3.h3_euler_step_bf16(lat_audio, st.v_audio, sa[s], sa[s + 1], audio_bf16, stream=stream)
+
+    def run(self, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, n_steps: int, stream=None):
+        """lat_*: fp32 latents at sigma = 1, updated in place; *_bf16: their
+        bf16 copies (the first step's transformer input), kept in step."""
+        sv = h3.h3_sigma_schedule(n_steps, self.shifts[0])
+        sa = h3.h3_sigma_schedule(n_steps, self.shifts[1])
+        for s in range(n_steps):
+            self.step(s, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, sv, sa, stream)
+
+    def launches_per_step(self) -> int:
+        st = self.st
+        return st.launches_per_step() - 2 - 7 + 7 * self.n_layers + 2

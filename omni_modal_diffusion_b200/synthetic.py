@@ -129,3 +129,28 @@ def random_rows(n_valid: int, k: int, seed: int) -> np.ndarray:
     rng = np.random.default_rng(seed)
     k = min(k, n_valid)
     return np.sort(rng.choice(n_valid, size=k, replace=False))
+
+
+def make_stack_inputs(w: Workload, n_layers: int, n_steps: int, seed: int | None = None) -> dict:
+    """Inputs of the layered sampler: per-block weights (list of dicts with
+    Wqkv, qn_w, kn_w, Wo, Wgu, Wd as in make_inputs), modulation
+    mod_all [n_steps][n_layers][3][6][D] float32 N(0, 0.1), and the initial
+    latents at sigma = 1 (float32 N(0, 1), not rounded: the sampler state is
+    fp32; the transformer reads its bf16 rounding)."""
+    rng = np.random.default_rng((7777 + w.index) if seed is None else seed)
+    blocks = []
+    for _ in range(n_layers):
+        blocks.append({
+            "Wqkv": bf16_round(_normal(rng, (3 * w.I, w.D), 0.02)),
+            "qn_w": bf16_round(_normal(rng, (w.head_dim,), 0.1, 1.0)),
+            "kn_w": bf16_round(_normal(rng, (w.head_dim,), 0.1, 1.0)),
+            "Wo": bf16_round(_normal(rng, (w.D, w.I), 0.02)),
+            "Wgu": bf16_round(_normal(rng, (2 * w.F, w.D), 0.02)),
+            "Wd": bf16_round(_normal(rng, (w.D, w.F), 0.02)),
+        })
+    return {
+        "blocks": blocks,
+        "mod_all": _normal(rng, (n_steps, n_layers, 3, 6, w.D), std=0.1),
+        "lat_video": _normal(rng, (w.T_lat, w.H_lat, w.W_lat, w.C_lat)),
+        "lat_audio": _normal(rng, (w.audio_channels, w.n_audio, w.C_audio)),
+    }

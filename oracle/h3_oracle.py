@@ -372,6 +372,43 @@ def head_unpack(x, ranges, W_vhead, W_ahead, t_lat, h_lat, w_lat, audio_channels
 
 
 # --------------------------------------------------------------------------
+# A12  the sampler loop
+# --------------------------------------------------------------------------
+
+def round_to_bf16(a):
+    """Nearest bfloat16 value (8 significant bits, ties to even), as float64:
+    the transformer reads its latent inputs in bf16, so the sampler loop
+    rounds the latent there, as the GPU path does."""
+    a = np.asarray(a, np.float64)
+    m, e = np.frexp(a)                       # a = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
+
+
+def sample(text, lat_video, lat_audio, io, blocks, mod_all, ranges, pos, n_heads, n_steps,
+           shift_video=12.0, shift_audio=3.0, head_dim=128, split=(32, 48, 48)):
+    """n_steps Euler steps of the flow sampler over a stack of blocks
+    [shouss §6; 0539 scheduler shifts]: each step packs and projects the
+    bf16-rounded latents, runs every block with its own modulation
+    mod_all[step][block], maps the result to per-modality velocities with the
+    head and moves each latent along its own shifted schedule; the text is a
+    condition and is never updated [shouss §5].  Returns the final latents."""
+    sv, sa = sigma_schedule(n_steps, shift_video), sigma_schedule(n_steps, shift_audio)
+    lv = np.asarray(lat_video, np.float64).copy()
+    la = np.asarray(lat_audio, np.float64).copy()
+    T, Hl, Wl, _ = lv.shape
+    ch, na, _ = la.shape
+    for s in range(n_steps):
+        x = embed(text, round_to_bf16(lv), round_to_bf16(la), io["W_text"], io["W_vid"], io["W_aud"], ranges)
+        for b, W in enumerate(blocks):
+            x = block_forward(x, mod_all[s][b], ranges, pos, W["Wqkv"], W["qn_w"], W["kn_w"], W["Wo"], W["Wgu"],
+                              W["Wd"], n_heads, head_dim, split)
+        vv, va = head_unpack(x, ranges, io["W_vhead"], io["W_ahead"], T, Hl, Wl, ch, na)
+        lv = euler_step(lv, vv, sv[s], sv[s + 1])
+        la = euler_step(la, va, sa[s], sa[s + 1])
+    return lv, la
+
+
+# --------------------------------------------------------------------------
 # A11  flow sampler
 # --------------------------------------------------------------------------
 

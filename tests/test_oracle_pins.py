@@ -430,3 +430,50 @@ def test_head_unpack_shapes_and_roundtrip():
     h = O.layernorm(x)
     s = r["start"][O.VIDEO]
     _pin_close(O.patchify(vv), O.linear(h[s:s + 12], Wv), 1e-12)
+
+
+# ---------------------------------------------------------------- A12
+
+def test_round_to_bf16_matches_library_conversion():
+    x = (np.random.default_rng(17).standard_normal(200000) * 7).astype(np.float32)
+    x[:6] = [0.0, -0.0, 1.0, -3.0e38, 2.5e-38, 1.00390625]      # 1 + 2^-8: a tie, rounds to even (1.0)
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.round_to_bf16(x), ref)
+
+
+def test_sampler_with_zero_head_keeps_latents_and_text():
+    """A head with zero weights gives zero velocity: every Euler step leaves
+    the latents exactly unchanged, for any schedule."""
+    w = S.WORKLOADS["tiny"]
+    inp = S.make_inputs(w)
+    st = S.make_stack_inputs(w, 2, 3)
+    io = dict(inp)
+    io["W_vhead"] = np.zeros_like(inp["W_vhead"])
+    io["W_ahead"] = np.zeros_like(inp["W_ahead"])
+    t, i, j = O.token_grid(w.T_lat, w.H_lat, w.W_lat)
+    r = O.pack_ranges(w.n_text, w.audio_channels * w.n_audio, t * i * j)
+    pos = O.positions(r, t, i, j, w.audio_channels, w.n_audio)
+    lv, la = O.sample(inp["text"], st["lat_video"], st["lat_audio"], io, st["blocks"], st["mod_all"], r, pos, w.H, 3)
+    assert np.array_equal(lv, st["lat_video"].astype(np.float64))
+    assert np.array_equal(la, st["lat_audio"].astype(np.float64))
+
+
+def test_sampler_one_step_is_euler_of_the_block_stack():
+    """One step from sigma 1 to 0 moves each latent by minus its velocity
+    (sum of sigma differences = -1), with the velocity of the block stack on
+    the bf16-rounded latents."""
+    w = S.WORKLOADS["tiny"]
+    inp = S.make_inputs(w)
+    st = S.make_stack_inputs(w, 2, 1)
+    t, i, j = O.token_grid(w.T_lat, w.H_lat, w.W_lat)
+    r = O.pack_ranges(w.n_text, w.audio_channels * w.n_audio, t * i * j)
+    pos = O.positions(r, t, i, j, w.audio_channels, w.n_audio)
+    lv, la = O.sample(inp["text"], st["lat_video"], st["lat_audio"], inp, st["blocks"], st["mod_all"], r, pos, w.H, 1)
+    x = O.embed(inp["text"], O.round_to_bf16(st["lat_video"]), O.round_to_bf16(st["lat_audio"]), inp["W_text"],
+                inp["W_vid"], inp["W_aud"], r)
+    for b in range(2):
+        x = O.block_forward(x, st["mod_all"][0][b], r, pos, n_heads=w.H, **st["blocks"][b])
+    vv, va = O.head_unpack(x, r, inp["W_vhead"], inp["W_ahead"], w.T_lat, w.H_lat, w.W_lat, w.audio_channels,
+                           w.n_audio)
+    _pin_close(lv, st["lat_video"] - vv, 1e-12)
+    _pin_close(la, st["lat_audio"] - va, 1e-12)
