@@ -51,6 +51,7 @@ struct GemmProblem {
   int N_b_rows;   // rows of B (for the tensor map extent)
   int M, K;
   int n_tiles;    // number of 256-wide (or 128-pair for SwiGLU) column tiles
+  int group_m;    // tile order: bands of group_m row tiles sweep all column tiles (L2 reuse of A)
   int b_second_half_off;  // SwiGLU: row offset of the "up" half in B (= F); else 128
   GemmEpilogue epi;
 };
