@@ -67,7 +67,13 @@ def bytes_per_call(w, L, Lp):
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel on
 # this workload, valid for the kernel as it was when captured; None once the
 # kernel changes (see profiles/).
-TRAFFIC = {}
+TRAFFIC = {
+    # mean over the block's QKV, out-projection, FFN gate/up and FFN down
+    # launches (6.050 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel"): 1.513e9,
+    # profiles/attention_tc_kernel_768sq_2s.md
+    ("768sq_2s", "attention_tc_kernel"): 0.435e9,
+}
 
 
 class ClockSampler:
@@ -263,9 +269,11 @@ def run_ours(args, w):
     gemm_tf = sum(fl[c] for c in gemm_calls) / (gemm_ms / 1e3) / 1e12
     attn_tf = tensor_calls["h3_attention"]
     kernels = {"gemm_tc_kernel": {"ms_per_step": round(gemm_ms, 4), "launches_per_step": 4,
-                                  "tflops": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4)},
+                                  "tflops": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4),
+                                  "traffic_per_launch": TRAFFIC.get((w.name, "gemm_tc_kernel"))},
                "attention_tc_kernel": {"ms_per_step": round(per_call["h3_attention"], 4), "launches_per_step": 1,
-                                       "tflops": round(attn_tf, 1), "frac": round(attn_tf / peak_tf, 4)}}
+                                       "tflops": round(attn_tf, 1), "frac": round(attn_tf / peak_tf, 4),
+                                       "traffic_per_launch": TRAFFIC.get((w.name, "attention_tc_kernel"))}}
     dominant = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     block_flops = sum(fl.values())
     block_ms = sum(per_call[c] for c in ("h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
