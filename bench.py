@@ -126,6 +126,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank timings over the process group (the
+    slowest rank sets a multi-GPU time).  Works for any backend; identity
+    without an initialised group."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Units of all ranks per second when every rank processes its own
+    units_per_rank in ms_per_step (the max over ranks)."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -241,21 +259,16 @@ def run_ours(args, w):
     ms_e2e = e0.elapsed_time(e1)
 
     # max over ranks
-    vals = torch.tensor([ms_total, ms_e2e], device=dev, dtype=torch.float64)
+    ms_total, ms_e2e = max_over_ranks([ms_total, ms_e2e], device=dev)
+    per_call = dict(zip(calls, max_over_ranks([per_call[c] for c in calls], device=dev)))
     if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total, ms_e2e = vals.tolist()
-    per_call_t = torch.tensor([per_call[c] for c in calls], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(per_call_t, op=dist.ReduceOp.MAX)
         dist.destroy_process_group()
-    per_call = dict(zip(calls, per_call_t.tolist()))
     if rank != 0:
         return None
 
     ms_step = ms_total / args.steps
-    value = world * L / (ms_step / 1e3)
-    e2e_value = world * L / (ms_e2e / args.steps / 1e3)
+    value = job_throughput(world, L, ms_step)
+    e2e_value = job_throughput(world, L, ms_e2e / args.steps)
     peaks = _peaks()
     fl = flops_per_call(w, L)
     by = bytes_per_call(w, L, Lp)
