@@ -68,9 +68,6 @@ def bytes_per_call(w, L, Lp):
 # this workload, valid for the kernel as it was when captured; None once the
 # kernel changes (see profiles/).
 TRAFFIC = {
-    # mean over the block's QKV, out-projection, FFN gate/up and FFN down
-    # launches (6.050 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel"): 1.513e9,
     # profiles/attention_tc_kernel_768sq_2s.md
     ("768sq_2s", "attention_tc_kernel"): 0.435e9,
 }
@@ -274,9 +271,10 @@ def run_ours(args, w):
     by = bytes_per_call(w, L, Lp)
     tensor_calls = {c: fl[c] / (per_call[c] / 1e3) / 1e12 for c in fl}
     peak_tf = peaks["bf16_tflops_sustained"]
-    # Kernels: gemm_tc_kernel runs the QKV, out-projection, FFN gate/up and FFN
-    # down launches (the embed/head launches add < 0.4% of its FLOPs and are
-    # not timed separately); attention_tc_kernel is one launch per step.
+    # Kernels: the tcgen05 GEMM (gemm_tc2_kernel, CTA pairs, for QKV and the
+    # out-projection; gemm_tc_kernel for the FFN's gate/up and down) runs the
+    # block's four GEMM launches (the embed/head launches add < 0.4% of its
+    # FLOPs and are not timed separately); attention_tc_kernel is one launch.
     gemm_calls = ("h3_qkv_qknorm_mrope", "h3_gated_residual", "h3_ffn_swiglu")
     gemm_ms = sum(per_call[c] for c in gemm_calls)
     gemm_tf = sum(fl[c] for c in gemm_calls) / (gemm_ms / 1e3) / 1e12

@@ -356,6 +356,169 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cta_group::2): a cluster of two CTAs computes a 256 x 256
+// tile; CTA r stages A rows [128 r, 128 r + 128) and B rows [128 r, 128 r + 128)
+// of the tile (for SwiGLU: r = 0 the gate rows, r = 1 the up rows) in its own
+// shared memory, and the leader CTA (rank 0) issues M = 256 MMAs that read
+// both CTAs' operands and leave each CTA's 128 result rows in its own TMEM.
+// Per CTA this stages 32 KB per 64-deep K step instead of 48 KB.
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = 128 * BK * 2;             // 16 KB
+constexpr int P_B_BYTES = 128 * BK * 2;             // 16 KB (half of the 256 columns)
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 512;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmProblem p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + P_STAGES * P_A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* tfull = empty + P_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  float* freq = reinterpret_cast<float*>(tmem_slot + 4);
+  uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const GemmEpilogue& e = p.epi;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);    // the leader's producer arrives (+ both CTAs' bytes)
+      mbar_init(&empty[s], 1);   // the leader's MMA commit, delivered to both CTAs
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);   // the leader's commit, delivered to both CTAs
+      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA (leader's copy used)
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (e.mode == EPI_QKV && threadIdx.x >= 64 && threadIdx.x < 128) {
+    const int i = threadIdx.x - 64;
+    const int pt = e.rope_t / 2, ph = e.rope_h / 2;
+    int ax, i_sec, d_sec;
+    if (i < pt) { ax = 0; i_sec = i; d_sec = e.rope_t; }
+    else if (i < pt + ph) { ax = 1; i_sec = i - pt; d_sec = e.rope_h; }
+    else { ax = 2; i_sec = i - pt - ph; d_sec = e.rope_w; }
+    freq[i] = powf(e.theta, -2.0f * (float)i_sec / (float)d_sec);
+    axis_of_pair[i] = (uint8_t)ax;
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int m_pairs = (p.M + 255) / 256;
+  const int num_tiles = m_pairs * p.n_tiles;
+  const int num_kb = (p.K + BK - 1) / BK;
+  const bool swiglu = e.mode == EPI_SWIGLU;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += n_pairs) {
+        int mt, nt;
+        tile_coords(t, m_pairs, p.n_tiles, p.group_m, mt, nt);
+        const int arow = mt * 256 + (int)rank * 128;
+        const int brow = nt * (swiglu ? 128 : 256) + (int)rank * p.b_second_half_off;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+          const uint32_t fb = leader_full0 + stage * 8;
+          tma_load_2d_pair(smA + stage * P_A_BYTES, &tmA, fb, kb * BK, arow);
+          tma_load_2d_pair(smB + stage * P_B_BYTES, &tmB, fb, kb * BK, brow);
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(256, 256, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += n_pairs) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smA + stage * P_A_BYTES);
+          const uint32_t b_addr = smem_u32(smB + stage * P_B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          umma_commit_pair(&empty[stage]);
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
+        }
+        umma_commit_pair(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles; t += n_pairs) {
+      int mt, nt;
+      tile_coords(t, m_pairs, p.n_tiles, p.group_m, mt, nt);
+      bool ok = mbar_wait(&tfull[acc], acc_phase);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int m = mt * 256 + (int)rank * 128 + row_in_tile;
+      switch (e.mode) {
+        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN); break;
+        case EPI_GATED_RESID: epi_gated_resid(e, tb, m, nt * BN); break;
+        case EPI_SWIGLU: epi_swiglu(e, tb, m, nt); break;
+        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair); break;
+        case EPI_UNPATCH: epi_unpatch(e, tb, m, nt * BN); break;
+        default: break;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + acc * 8);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no MMA of the pair is in flight and no remote arrival pending
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -428,6 +591,32 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     const long long panel = 128ll * p.K * 2;
     long long g = H3_GEMM_BAND_BYTES / (panel > 0 ? panel : 1);
     q.group_m = (int)(g < 1 ? 1 : (g > m_tiles ? m_tiles : g));
+  }
+#ifndef H3_GEMM_PAIR
+#define H3_GEMM_PAIR 1
+#endif
+  // Per call (measured on B200 at 7,904 / 32,160 tokens): the pair kernel
+  // takes the out-projection from 0.49 / 1.96 ms to 0.45 / 1.79 ms and the
+  // QKV GEMM from 1.30 / 5.33 ms to 1.27 / 5.24 ms, but is up to 5% slower
+  // on the FFN's gate/up and down GEMMs at 32,160 tokens, so callers choose.
+  if (H3_GEMM_PAIR && p.pair == 1 && p.M > 128) {
+    static bool attr2_set = false;
+    if (!attr2_set) {
+      cudaError_t err = cudaFuncSetAttribute(gemm_detail::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             gemm_detail::P_SMEM_BYTES);
+      if (err != cudaSuccess) return err;
+      attr2_set = true;
+    }
+    const int m_pairs = (p.M + 255) / 256;
+    GemmProblem q2 = q;
+    if (p.group_m <= 0) q2.group_m = (q.group_m + 1) / 2 > 0 ? (q.group_m + 1) / 2 : 1;
+    if (q2.group_m > m_pairs) q2.group_m = m_pairs;
+    const int pair_tiles = m_pairs * p.n_tiles;
+    const int max_pairs = num_sms() / 2;
+    const int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
+    gemm_detail::gemm_tc2_kernel<<<2 * pairs, gemm_detail::NUM_THREADS, gemm_detail::P_SMEM_BYTES, stream>>>(
+        tmA, tmB, q2);
+    return cudaGetLastError();
   }
   const int grid = tiles < num_sms() ? tiles : num_sms();
   gemm_tc_kernel<<<grid, gemm_detail::NUM_THREADS, gemm_detail::SMEM_BYTES, stream>>>(tmA, tmB, q);

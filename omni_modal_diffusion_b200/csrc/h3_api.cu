@@ -224,6 +224,7 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
   H3_REQUIRE_PTR(v);
   const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
   GemmProblem p = gemm_base(xm, D, Lp, D, Wqkv, D, 3 * I, (3 * I + 255) / 256);
+  p.pair = 1;
   GemmEpilogue& ep = p.epi;
   ep.mode = EPI_QKV;
   ep.M = Lp;
@@ -286,6 +287,7 @@ int h3_gated_residual(const h3_dims* dims, const h3_ranges* ranges, float* x, co
   H3_REQUIRE_PTR(mod);
   const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
   GemmProblem p = gemm_base(o, I, Lp, I, Wo, I, D, (D + 255) / 256);
+  p.pair = 1;
   p.epi.mode = EPI_GATED_RESID;
   p.epi.M = Lp;
   p.epi.N = D;

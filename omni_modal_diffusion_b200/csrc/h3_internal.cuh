@@ -52,6 +52,7 @@ struct GemmProblem {
   int M, K;
   int n_tiles;    // number of 256-wide (or 128-pair for SwiGLU) column tiles
   int group_m;    // tile order: bands of group_m row tiles sweep all column tiles (L2 reuse of A)
+  int pair;       // 1: CTA-pair kernel (256 x 256 tiles over two SMs) when M > 128; 0: one CTA per tile
   int b_second_half_off;  // SwiGLU: row offset of the "up" half in B (= F); else 128
   GemmEpilogue epi;
 };
