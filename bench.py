@@ -68,6 +68,9 @@ def bytes_per_call(w, L, Lp):
 # this workload, valid for the kernel as it was when captured; None once the
 # kernel changes (see profiles/).
 TRAFFIC = {
+    # mean over the block's QKV, out-projection, FFN gate/up and FFN down
+    # launches (6.090 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel"): 1.523e9,
     # profiles/attention_tc_kernel_768sq_2s.md
     ("768sq_2s", "attention_tc_kernel"): 0.435e9,
 }

@@ -72,13 +72,17 @@ __global__ void zero_rows_kernel(float* __restrict__ x, long first, long last, i
 }
 
 // ------------------------------------------------------------ LN + modulate
-// One CTA of 256 threads per row; each thread keeps up to VPT float4 of the
-// row in registers.  Two-pass mean/variance in fp32 (biased variance),
-// h = (x - mu) / sqrt(var + eps), out = h * (1 + scale_m) + shift_m with m the
-// modality of the row's token range ("MiniMax-H3: native joint audio-video
-// generation" (note.shouss.top) §3, §3.1).  mod == nullptr: plain LN.
-constexpr int LN_THREADS = 256;
-constexpr int LN_VPT = 8;  // up to 8192 columns
+// One CTA per row; thread i keeps float4 elements i, i + T, i + 2T, ... of the
+// row in registers (up to LN_VPT of them).  Two-pass mean/variance in fp32
+// (biased variance), h = (x - mu) / sqrt(var + eps), out = h * (1 + scale_m) +
+// shift_m with m the modality of the row's token range ("MiniMax-H3: native
+// joint audio-video generation" (note.shouss.top) §3, §3.1).  mod == nullptr:
+// plain LN.  Stores are 8 bytes (4 bf16) per float4 read.
+#ifndef H3_LN_THREADS
+#define H3_LN_THREADS 256
+#endif
+constexpr int LN_THREADS = H3_LN_THREADS;
+constexpr int LN_VPT = (2048 + LN_THREADS - 1) / LN_THREADS;  // up to 8192 columns
 
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
@@ -89,7 +93,7 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   __syncthreads();
   float t = 0.f;
 #pragma unroll
-  for (int i = 0; i < LN_THREADS / 32; ++i) t += red[i];
+  for (int i = 0; i < (LN_THREADS + 31) / 32; ++i) t += red[i];
   return t;
 }
 
@@ -97,7 +101,7 @@ __global__ void __launch_bounds__(LN_THREADS) ln_modulate_kernel(const float* __
                                                                   const float* __restrict__ mod, int branch,
                                                                   RangeArgs rg, int L, int D, float eps,
                                                                   bf16* __restrict__ out) {
-  __shared__ float red[LN_THREADS / 32];
+  __shared__ float red[(LN_THREADS + 31) / 32];
   const int row = blockIdx.x;
   const int nv = D / 4;
   bf16* orow = out + (long)row * D;
