@@ -320,13 +320,10 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
                     uint32_t box_rows);
 
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t err = cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           attn_detail::SMEM_BYTES);
-    if (err != cudaSuccess) return err;
-    attr_set = true;
-  }
+  static unsigned long long attr_done = 0;
+  cudaError_t aerr =
+      ensure_smem_attr(reinterpret_cast<const void*>(attention_tc_kernel), attn_detail::SMEM_BYTES, &attr_done);
+  if (aerr != cudaSuccess) return aerr;
   CUtensorMap tq, tk, tv;
   const uint64_t rows = (uint64_t)p.H * p.L_pad;
   if (!make_tmap_bf16(&tq, p.q, rows, 128, 128, 128)) return cudaErrorInvalidValue;

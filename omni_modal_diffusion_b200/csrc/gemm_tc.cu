@@ -554,24 +554,34 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 }
 
 int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+    cache[dev] = n > 0 ? n : 148;
   }
-  return n;
+  return cache[dev];
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* done_mask) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (*done_mask & bit) return cudaSuccess;
+  err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) *done_mask |= bit;
+  return err;
 }
 
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
   if (p.M <= 0) return cudaSuccess;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t err = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_detail::SMEM_BYTES);
-    if (err != cudaSuccess) return err;
-    attr_set = true;
-  }
+  static unsigned long long attr_done = 0;
+  cudaError_t aerr = ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel), gemm_detail::SMEM_BYTES, &attr_done);
+  if (aerr != cudaSuccess) return aerr;
   CUtensorMap tmA, tmB;
   if (!make_tmap_bf16(&tmA, p.A, (uint64_t)p.M, (uint64_t)p.K, (uint64_t)p.lda, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tmB, p.B, (uint64_t)p.N_b_rows, (uint64_t)p.K, (uint64_t)p.ldb, 128))
@@ -600,13 +610,10 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
   // QKV GEMM from 1.30 / 5.33 ms to 1.27 / 5.24 ms, but is up to 5% slower
   // on the FFN's gate/up and down GEMMs at 32,160 tokens, so callers choose.
   if (H3_GEMM_PAIR && p.pair == 1 && p.M > 128) {
-    static bool attr2_set = false;
-    if (!attr2_set) {
-      cudaError_t err = cudaFuncSetAttribute(gemm_detail::gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             gemm_detail::P_SMEM_BYTES);
-      if (err != cudaSuccess) return err;
-      attr2_set = true;
-    }
+    static unsigned long long attr2_done = 0;
+    cudaError_t err2 = ensure_smem_attr(reinterpret_cast<const void*>(gemm_detail::gemm_tc2_kernel),
+                                        gemm_detail::P_SMEM_BYTES, &attr2_done);
+    if (err2 != cudaSuccess) return err2;
     const int m_pairs = (p.M + 255) / 256;
     GemmProblem q2 = q;
     if (p.group_m <= 0) q2.group_m = (q.group_m + 1) / 2 > 0 ? (q.group_m + 1) / 2 : 1;

@@ -84,4 +84,8 @@ cudaError_t launch_euler(float* lat, const float* vel, long long n, float dsigma
 
 int num_sms();
 
+// cudaFuncSetAttribute(func, MaxDynamicSharedMemorySize, bytes) once per
+// device (function attributes are per device context).
+cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* done_mask);
+
 }  // namespace h3
