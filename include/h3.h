@@ -247,6 +247,13 @@ int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, con
 int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, h3_bf16* lat_bf16,
                        void* stream);
 
+/* Diagnostic for failure detection: one device thread waits, with the given
+ * limit (nanoseconds, at most 10 s), on an mbarrier that nothing arrives on.
+ * The wait gives up and records code 1 in the device error word exactly as a
+ * stalled pipeline wait would; h3_device_status then returns H3_ERR_TIMEOUT.
+ * Nothing faults and the context stays usable. */
+int h3_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* Synchronise `stream`, then report (and clear) the device error word that
  * bounded device-side waits set when they give up.  *code_out = 0 when no
  * wait failed.  Returns H3_ERR_TIMEOUT if one did, H3_ERR_CUDA on a CUDA

@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* s_full = bars + 9;    // [2] per query tile
   uint64_t* o_final = bars + 11;  // [2] per query tile
   uint64_t* p_full = bars + 13;   // [2 tiles][2 halves of the key tile]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* drain = bars + 17;    // the MMA issuer's last commit before teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&p_full[2 * s + 1], 4);
       mbar_init(&o_final[s], 1);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -113,6 +115,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_load_2d(sQ + HALF_BYTES, &tmQ, q_full, 64, row0 + qt0 * TILE);
       tma_load_2d(sQ + TILE_BYTES, &tmQ, q_full, 0, row0 + qt1 * TILE);
       tma_load_2d(sQ + TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, row0 + qt1 * TILE);
+      long long k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
         uint8_t* dk = sK + st * TILE_BYTES;
@@ -121,11 +124,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
         tma_load_2d(dk, &tmK, &k_full[st], 0, row0 + j * TILE);
         tma_load_2d(dk + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
+        ++k_issued;
         if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
         tma_load_2d(dv, &tmV, &v_full[st], 0, row0 + j * TILE);
         tma_load_2d(dv + HALF_BYTES, &tmV, &v_full[st], 64, row0 + j * TILE);
+        ++v_issued;
       }
+      // every load of this CTA has landed before it leaves
+      mbar_wait(q_full, 0);
+      drain_loads(k_full, 2, k_issued);
+      drain_loads(v_full, 2, v_issued);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -187,6 +196,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         umma_commit(&v_empty[j & 1]);
       }
+      drain_mmas(drain);
     }
   } else {
     const int t = (warp - 2) >> 2;  // query tile of this warpgroup

@@ -197,6 +197,16 @@ __global__ void euler_bf16_kernel(float* __restrict__ lat, const float* __restri
   }
 }
 
+// One thread waits on an mbarrier that nothing arrives on: the bounded wait
+// gives up after limit_ns and records its error code, like any stalled
+// pipeline wait in the tensor-core kernels.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait_limit(&bar, 0, limit_ns);
+}
+
 // The attention softmax's FMA-pipe exponential on an array (for checking it
 // against its error bound).
 __global__ void exp2_fma_pipe_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
@@ -254,6 +264,11 @@ cudaError_t launch_ln_modulate(const float* x, const float* mod, int branch, con
     rg.count[m] = rcount[m];
   }
   ln_modulate_kernel<<<L_pad, LN_THREADS, 0, stream>>>(x, mod, branch, rg, L, D, eps, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 1, 0, stream>>>(limit_ns);
   return cudaGetLastError();
 }
 

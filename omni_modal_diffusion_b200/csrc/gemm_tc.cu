@@ -223,7 +223,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
 
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 4);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      long long issued = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int mt, nt;
@@ -285,9 +288,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d(smA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, mt * BM);
           tma_load_2d(smB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * BK, b0);
           tma_load_2d(smB + stage * B_STAGE_BYTES + B_STAGE_BYTES / 2, &tmB, &full[stage], kb * BK, b1);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      drain_loads(full, STAGES, issued);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -318,6 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_commit(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
+      drain_mmas(drain);
     }
   } else {
     const int q = warp & 3;
@@ -381,7 +387,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   uint64_t* empty = full + P_STAGES;
   uint64_t* tfull = empty + P_STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
 
@@ -400,6 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tfull[a], 1);   // the leader's commit, delivered to both CTAs
       mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA (leader's copy used)
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -434,6 +442,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
       int stage = 0;
       uint32_t phase = 0;
+      long long issued = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += n_pairs) {
         int mt, nt;
@@ -446,9 +455,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb = leader_full0 + stage * 8;
           tma_load_2d_pair(smA + stage * P_A_BYTES, &tmA, fb, kb * BK, arow);
           tma_load_2d_pair(smB + stage * P_B_BYTES, &tmB, fb, kb * BK, brow);
+          ++issued;
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
       }
+      // the leader's full barriers count both CTAs' bytes: the leader waits
+      // for both, the peer CTA is held by the cluster barrier below
+      if (leader) drain_loads(full, P_STAGES, issued);
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
@@ -479,6 +492,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         umma_commit_pair(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
+      umma_commit_pair(drain);
+      mbar_wait(drain, 0);
     }
   } else {
     const int q = warp & 3;

@@ -456,6 +456,14 @@ int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream) {
   return ok();
 }
 
+int h3_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull)
+    return fail(H3_ERR_SHAPE, "h3_selftest_wait_timeout: limit must be in (0, 10 s]");
+  cudaError_t e = launch_wait_timeout_selftest((unsigned long long)limit_ns, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "h3_selftest_wait_timeout");
+  return ok();
+}
+
 int h3_device_status(void* stream, int* code_out) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: synchronize");

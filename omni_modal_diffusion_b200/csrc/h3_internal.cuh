@@ -77,6 +77,7 @@ cudaError_t launch_pack(const bf16* video, int T, int Hl, int Wl, int C_lat, int
                         uint8_t* mod_ids, float* x, int D, cudaStream_t stream);
 cudaError_t launch_ln_modulate(const float* x, const float* mod, int branch, const int* rstart, const int* rcount,
                                int L, int L_pad, int D, float eps, bf16* out, cudaStream_t stream);
+cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_fma_pipe(const float* x, float* y, long long n, cudaStream_t stream);
 cudaError_t launch_euler_bf16(float* lat, const float* vel, long long n, float dsigma, bf16* out,
                               cudaStream_t stream);

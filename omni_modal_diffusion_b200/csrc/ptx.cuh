@@ -78,6 +78,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// As mbar_wait with an explicit limit (used by the timeout self-test).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicCAS(&g_h3_device_error, 0, 1);
+      return false;
+    }
+  }
+}
+
 // Non-blocking probe of a phase (no suspension of the calling thread).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -291,6 +305,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------ exit paths
+// Before a CTA leaves (normally or after a wait gave up): wait, bounded, for
+// the last `stages` of the `issued` TMA stage loads that signal `full[]`
+// (stage k of the ring: barrier k % stages, phase parity (k / stages) & 1).
+// Loads already consumed have completed and pass at once.
+__device__ __forceinline__ void drain_loads(uint64_t* full, int stages, long long issued) {
+  for (long long k = issued > stages ? issued - stages : 0; k < issued; ++k)
+    if (!mbar_wait(&full[k % stages], (uint32_t)((k / stages) & 1))) return;
+}
+// Wait, bounded, until every MMA this thread issued has completed.
+__device__ __forceinline__ void drain_mmas(uint64_t* bar) {
+  umma_commit(bar);
+  mbar_wait(bar, 0);
+}
 
 // ------------------------------------------------------------ misc
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -25,7 +25,7 @@ EXPORTS = (
     "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention", "h3_gated_residual",
     "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
     "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_exp2_fma_pipe", "h3_block_forward",
-    "h3_euler_step_bf16",
+    "h3_euler_step_bf16", "h3_selftest_wait_timeout",
 )
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
 
@@ -90,6 +90,7 @@ def lib() -> ctypes.CDLL:
                                       ci, vp]),
             "h3_device_status": (ci, [vp, ctypes.POINTER(ci)]),
             "h3_set_wait_limit_ns": (ci, [ctypes.c_uint64]),
+            "h3_selftest_wait_timeout": (ci, [ctypes.c_uint64, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -241,6 +242,10 @@ def h3_device_status(stream=None) -> int:
     if rc not in (H3_OK, H3_ERR_TIMEOUT):
         _check(rc)
     return code.value
+
+
+def h3_selftest_wait_timeout(limit_ns: int, stream=None):
+    _check(lib().h3_selftest_wait_timeout(limit_ns, _stream(stream)))
 
 
 def h3_set_wait_limit_ns(ns: int):
