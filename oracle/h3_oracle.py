@@ -367,7 +367,7 @@ def head_unpack(x, ranges, W_vhead, W_ahead, t_lat, h_lat, w_lat, audio_channels
     sv, cv = ranges["start"][VIDEO], ranges["count"][VIDEO]
     sa, ca = ranges["start"][AUDIO], ranges["count"][AUDIO]
     v_video = unpatchify(linear(h[sv:sv + cv], W_vhead), t_lat, h_lat, w_lat)
-    v_audio = linear(h[sa:sa + ca], W_ahead).reshape(audio_channels, n_audio, -1)
+    v_audio = linear(h[sa:sa + ca], W_ahead).reshape(audio_channels, n_audio, np.asarray(W_ahead).shape[0])
     return v_video, v_audio
 
 
