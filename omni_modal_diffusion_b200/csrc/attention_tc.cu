@@ -49,6 +49,15 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #define H3_ATTN_SPLIT_P 0
 #endif
 constexpr int POLY_EVERY = H3_ATTN_POLY_EVERY;
+// How the MMA issuer waits: polling (1) or suspending try_wait (0).
+#ifndef H3_ATTN_MMA_SPIN
+#define H3_ATTN_MMA_SPIN 1
+#endif
+#if H3_ATTN_MMA_SPIN
+#define MMA_WAIT mbar_wait_spin
+#else
+#define MMA_WAIT mbar_wait
+#endif
 constexpr bool SPLIT_P = H3_ATTN_SPLIT_P != 0;
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -140,31 +149,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
       const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);  // V is MN-major (d contiguous)
-      const uint32_t q_addr = smem_u32(sQ);
+      // Shared-memory descriptors are computed once; an MMA then costs one
+      // 64-bit add (the start-address field is bits [0,14) in 16-byte units,
+      // and every offset below stays inside the 228 KB window).
+      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t v_desc = sdesc_sw128(smem_u32(sV), HALF_BYTES, 1024);
       // S_t = Q_t K_j^T into TMEM columns [256t, 256t + 128)
       auto issue_s = [&](int t, int j) {
-        const uint32_t k_addr = smem_u32(sK + (j & 1) * TILE_BYTES);
+        const uint64_t qd = q_desc + (uint64_t)((t * TILE_BYTES) >> 4);
+        const uint64_t kd = k_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(q_addr + t * TILE_BYTES + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k_addr + off, 16, 1024);
-          umma_bf16(tmem + t * 256, ad, bd, idesc_s, kk != 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+          umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
         }
         umma_commit(&s_full[t]);
       };
       // O_t += P_t V_j for keys [64 hf, 64 hf + 64), P_t (bf16, packed)
       // read from TMEM where S_t was
       auto issue_pv_half = [&](int t, int j, int hf) {
-        const uint32_t v_addr = smem_u32(sV + (j & 1) * TILE_BYTES);
+        const uint64_t vd = v_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = hf * 4 + k4;
-          const uint64_t bd = sdesc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024);
-          umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, bd, idesc_o, (j | kk) != 0 ? 1u : 0u);
+          umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
+                           (j | kk) != 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait_spin(q_full, 0) && mbar_wait_spin(&k_full[0], 0);
+      bool ok = MMA_WAIT(q_full, 0) && MMA_WAIT(&k_full[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
@@ -176,8 +189,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < 2 && ok; ++t) {
           for (int hf = 0; hf < 2; ++hf) {
             if (SPLIT_P || hf == 0) {
-              if (!mbar_wait_spin(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
-              if (t == 0 && hf == 0 && !mbar_wait_spin(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+              if (!MMA_WAIT(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
+              if (t == 0 && hf == 0 && !MMA_WAIT(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
               tc_fence_after();
             }
             issue_pv_half(t, j, hf);
@@ -185,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
           if (more) {
             if (t == 0) {
-              if (!mbar_wait_spin(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
+              if (!MMA_WAIT(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
               tc_fence_after();
             }
             issue_s(t, j + 1);
