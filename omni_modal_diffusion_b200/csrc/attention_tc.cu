@@ -7,7 +7,7 @@
 // One CTA per (pair of 128-query tiles, head); the two query tiles share the
 // K/V stream and ping-pong on the tensor core:
 //   Warp 0     TMA producer: both Q tiles once, K/V tiles through a 2-stage ring.
-//   Warp 1     TMEM owner and MMA issuer, in the order
+//   Warp 1     TMEM owner and MMA issuer (the whole warp, converged), in the order
 //              S0_0 S1_0 | PV0_0 S0_1 | PV1_0 S1_1 | PV0_1 S0_2 | ...
 //              so that while one softmax warpgroup works on its S tile the
 //              tensor core runs the other tile's PV and next S.
@@ -54,9 +54,9 @@ constexpr int POLY_EVERY = H3_ATTN_POLY_EVERY;
 #define H3_ATTN_MMA_SPIN 1
 #endif
 #if H3_ATTN_MMA_SPIN
-#define MMA_WAIT mbar_wait_spin
+#define MMA_WAIT_WARP mbar_wait_spin_warp
 #else
-#define MMA_WAIT mbar_wait
+#define MMA_WAIT_WARP mbar_wait_warp
 #endif
 constexpr bool SPLIT_P = H3_ATTN_SPLIT_P != 0;
 
@@ -146,71 +146,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_loads(v_full, 2, v_issued);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-      const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);  // V is MN-major (d contiguous)
-      // Shared-memory descriptors are computed once; an MMA then costs one
-      // 64-bit add (the start-address field is bits [0,14) in 16-byte units,
-      // and every offset below stays inside the 228 KB window).
-      const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
-      const uint64_t v_desc = sdesc_sw128(smem_u32(sV), HALF_BYTES, 1024);
-      // S_t = Q_t K_j^T into TMEM columns [256t, 256t + 128)
-      auto issue_s = [&](int t, int j) {
-        const uint64_t qd = q_desc + (uint64_t)((t * TILE_BYTES) >> 4);
-        const uint64_t kd = k_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
+    // The whole warp runs the issue loop, converged; one elected lane issues.
+    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);  // V is MN-major (d contiguous)
+    // Shared-memory descriptors are computed once; an MMA then costs one
+    // 64-bit add (the start-address field is bits [0,14) in 16-byte units,
+    // and every offset below stays inside the 228 KB window).
+    const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t v_desc = sdesc_sw128(smem_u32(sV), HALF_BYTES, 1024);
+    // S_t = Q_t K_j^T into TMEM columns [256t, 256t + 128)
+    auto issue_s = [&](int t, int j) {
+      const uint64_t qd = q_desc + (uint64_t)((t * TILE_BYTES) >> 4);
+      const uint64_t kd = k_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-          umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
-        }
-        umma_commit(&s_full[t]);
-      };
-      // O_t += P_t V_j for keys [64 hf, 64 hf + 64), P_t (bf16, packed)
-      // read from TMEM where S_t was
-      auto issue_pv_half = [&](int t, int j, int hf) {
-        const uint64_t vd = v_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+        umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[t]);
+    };
+    // O_t += P_t V_j for keys [64 hf, 64 hf + 64), P_t (bf16, packed)
+    // read from TMEM where S_t was
+    auto issue_pv_half = [&](int t, int j, int hf) {
+      const uint64_t vd = v_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int kk = hf * 4 + k4;
-          umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
-                           (j | kk) != 0 ? 1u : 0u);
-        }
-      };
-      bool ok = MMA_WAIT(q_full, 0) && MMA_WAIT(&k_full[0], 0);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit(&k_empty[0]);
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = hf * 4 + k4;
+        umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
+                         (j | kk) != 0 ? 1u : 0u);
       }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const bool more = j + 1 < nkv;
-        for (int t = 0; t < 2 && ok; ++t) {
-          for (int hf = 0; hf < 2; ++hf) {
-            if (SPLIT_P || hf == 0) {
-              if (!MMA_WAIT(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
-              if (t == 0 && hf == 0 && !MMA_WAIT(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
-              tc_fence_after();
-            }
-            issue_pv_half(t, j, hf);
-          }
-          if (!ok) break;
-          if (more) {
-            if (t == 0) {
-              if (!MMA_WAIT(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
-              tc_fence_after();
-            }
-            issue_s(t, j + 1);
-            if (t == 1) umma_commit(&k_empty[(j + 1) & 1]);
-          } else {
-            umma_commit(&o_final[t]);
-          }
-        }
-        umma_commit(&v_empty[j & 1]);
-      }
-      drain_mmas(drain);
+    };
+    bool ok = MMA_WAIT_WARP(q_full, 0) && MMA_WAIT_WARP(&k_full[0], 0);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+      umma_commit(&k_empty[0]);
     }
+    for (int j = 0; j < nkv && ok; ++j) {
+      const bool more = j + 1 < nkv;
+      for (int t = 0; t < 2 && ok; ++t) {
+        for (int hf = 0; hf < 2; ++hf) {
+          if (SPLIT_P || hf == 0) {
+            if (!MMA_WAIT_WARP(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
+            if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_pv_half(t, j, hf);
+        }
+        if (!ok) break;
+        if (more) {
+          if (t == 0) {
+            if (!MMA_WAIT_WARP(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_s(t, j + 1);
+          if (t == 1) umma_commit(&k_empty[(j + 1) & 1]);
+        } else {
+          umma_commit(&o_final[t]);
+        }
+      }
+      umma_commit(&v_empty[j & 1]);
+    }
+    drain_mmas(drain);
   } else {
     const int t = (warp - 2) >> 2;  // query tile of this warpgroup
     const int qw = warp & 3;        // TMEM lane quarter this warp may access

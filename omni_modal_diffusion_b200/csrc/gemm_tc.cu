@@ -295,36 +295,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_loads(full, STAGES, issued);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN, false);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
+    // The whole warp runs the issue loop, converged; one elected lane issues.
+    const uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+    // descriptors computed once; per MMA only the start address moves
+    // (16-byte units: a 32-byte K step is +2)
+    const uint64_t a_desc0 = sdesc_sw128(smem_u32(smA), 16, 1024);
+    const uint64_t b_desc0 = sdesc_sw128(smem_u32(smB), 16, 1024);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smA + stage * A_STAGE_BYTES);
-          const uint32_t b_addr = smem_u32(smB + stage * B_STAGE_BYTES);
+        const uint64_t ad = a_desc0 + (uint64_t)((stage * A_STAGE_BYTES) >> 4);
+        const uint64_t bd = b_desc0 + (uint64_t)((stage * B_STAGE_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1; }
-        }
-        umma_commit(&tfull[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        for (int kk = 0; kk < BK / 16; ++kk)
+          umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
-      drain_mmas(drain);
+      umma_commit(&tfull[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    drain_mmas(drain);
   } else {
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
@@ -464,28 +464,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       if (leader) drain_loads(full, P_STAGES, issued);
     }
   } else if (warp == 1) {
-    if (leader && lane == 0) {
+    if (leader) {
+      // The leader's whole warp runs the issue loop, converged; one elected lane issues.
       const uint32_t idesc = idesc_bf16_f32(256, 256, false);
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(smA), 16, 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(smB), 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += n_pairs) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) break;
+        if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
+          if (!mbar_wait_warp(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smA + stage * P_A_BYTES);
-          const uint32_t b_addr = smem_u32(smB + stage * P_B_BYTES);
+          const uint64_t ad = a_desc0 + (uint64_t)((stage * P_A_BYTES) >> 4);
+          const uint64_t bd = b_desc0 + (uint64_t)((stage * P_B_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_addr + kk * 32, 16, 1024);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
           umma_commit_pair(&empty[stage]);
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }

@@ -122,6 +122,15 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Warp-uniform forms of the bounded waits, for warps that stay converged
+// (the MMA-issuing warps): every lane polls, and the warp agrees on the result.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+__device__ __forceinline__ bool mbar_wait_spin_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity));
+}
+
 // ------------------------------------------------------------ clusters (CTA pairs)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -205,55 +214,71 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 }
 // D (M = 256 rows: 128 in each CTA's TMEM) (+)= A * B^T, A rows split across
 // the pair, B columns split across the pair (same shared-memory offsets).
+// Warp-collective (see umma_bf16).
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+      "elect.sync l|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive once on the mbarrier at the same offset in both CTAs of the pair
-// when the pair's prior MMAs have completed.
+// when the pair's prior MMAs have completed.  Warp-collective.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+      "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
+      "elect.sync l|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}\n" ::"r"(
           smem_u32(bar)),
       "h"((uint16_t)3)
       : "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.  Issued by
-// one thread.  accumulate == 0 overwrites D.
+// The tcgen05.mma / tcgen05.commit helpers are warp-collective: all 32 lanes
+// of a converged warp call them with the same operands and one lane, picked
+// by elect.sync (always the lowest, so every MMA and the commits that track
+// them come from the same thread), issues the instruction.  A converged
+// issuing warp lets the compiler keep the descriptors in uniform registers;
+// issuing from inside a one-lane branch costs tens of cycles per MMA.
+//
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate;
+// accumulate == 0 overwrites D.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+      "elect.sync l|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]: A (M x 16 bf16 per instruction) is read
 // from TMEM, row m in lane m, two bf16 packed per 32-bit column.
+// Warp-collective.
 __device__ __forceinline__ void umma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                                  uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 l;\n\t"
+      "elect.sync l|e, 0xffffffff;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// Arrive once on `bar` when every previously issued tcgen05.mma of this thread
-// has completed.
+// Arrive once on `bar` when every previously issued tcgen05.mma of the
+// electing thread has completed.  Warp-collective.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .b32 l;\n\t"
+      "elect.sync l|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(smem_u32(bar))
+      : "memory");
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
@@ -315,9 +340,11 @@ __device__ __forceinline__ void drain_loads(uint64_t* full, int stages, long lon
   for (long long k = issued > stages ? issued - stages : 0; k < issued; ++k)
     if (!mbar_wait(&full[k % stages], (uint32_t)((k / stages) & 1))) return;
 }
-// Wait, bounded, until every MMA this thread issued has completed.
+// Wait, bounded, until every MMA this warp issued has completed.
+// Warp-collective.
 __device__ __forceinline__ void drain_mmas(uint64_t* bar) {
   umma_commit(bar);
+  __syncwarp();
   mbar_wait(bar, 0);
 }
 
