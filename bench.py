@@ -69,10 +69,10 @@ def bytes_per_call(w, L, Lp):
 # kernel changes (see profiles/).
 TRAFFIC = {
     # mean over the block's QKV, out-projection, FFN gate/up and FFN down
-    # launches (6.090 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel"): 1.523e9,
+    # launches (6.203 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel"): 1.551e9,
     # profiles/attention_tc_kernel_768sq_2s.md
-    ("768sq_2s", "attention_tc_kernel"): 0.435e9,
+    ("768sq_2s", "attention_tc_kernel"): 0.4355e9,
 }
 
 
