@@ -206,11 +206,11 @@ int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x,
  * [shouss] §5, §6).  lat, vel: fp32 device arrays of n elements. */
 int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream);
 
-/* Diagnostic: y[i] = 2^x[i] computed the way h3_attention computes a quarter
- * of its softmax exponentials on full key tiles, on the FMA pipe instead of
- * the MUFU unit: x clamped to >= -125, x = j + f with j = rint(x), 2^f from a
- * cubic (max relative error 7.5e-5 for x in [-125, 64]), 2^j added to the
- * exponent.  x, y: fp32 device arrays of n elements. */
+/* Diagnostic: y[i] = 2^x[i] on the FMA pipe instead of the MUFU unit, the
+ * form h3_attention can take for part of its softmax exponentials (a build
+ * option, off by default): x clamped to >= -125, x = j + f with j = rint(x),
+ * 2^f from a cubic (max relative error 7.5e-5 for x in [-125, 64]), 2^j added
+ * to the exponent.  x, y: fp32 device arrays of n elements. */
 int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream);
 
 /* Block weights and scratch buffers for h3_block_forward (all device
@@ -263,6 +263,94 @@ int h3_device_status(void* stream, int* code_out);
 /* Set the time limit (nanoseconds, > 0) of every device-side wait for
  * kernels launched afterwards on the current device (default 2 s). */
 int h3_set_wait_limit_ns(uint64_t ns);
+
+/* ------------------------------------------------------------------------
+ * FP8 (e4m3) GEMMs.  The pages report community FP8 / INT4 quantisations of
+ * the trunk ("H3's omni-modal ambition" (0539edu.com), ecosystem paragraph)
+ * and fix no format; these entry points take the block's four GEMMs to e4m3
+ * tensor-core MMAs (tcgen05 kind::f8f6f4, fp32 accumulate) with this scheme:
+ *   - e4m3 is the OCP OFP8 E4M3 format (bias 7, 3 mantissa bits, largest
+ *     finite 448, no infinities); encoding rounds to nearest, ties to even,
+ *     saturating to +-448, sign bit kept (h3_e4m3 holds one code).
+ *   - Row scaling: amax = max |row|; rscale = 448 / amax and scale =
+ *     amax / 448 (IEEE fp32 divisions); code = e4m3(row * rscale) with the
+ *     product rounded to fp32; a zero row has scale 0 and codes 0.
+ *   - Activations carry one scale per token (row), weights one per output
+ *     channel (row of the [out][in] weight).  A GEMM then computes
+ *     acc[m][n] * a_scale[m] * b_scale[n] and applies the same fused
+ *     epilogue as its bf16 counterpart.
+ * Attention stays bf16.  Code matrices are row-major bytes; every row length
+ * is a multiple of 16 bytes as for the bf16 calls (D % 64, I, F % 128). */
+typedef uint8_t h3_e4m3;
+
+/* Row quantisation of a bf16 matrix (weights offline; activations between
+ * calls).  in [rows][cols] with row stride ld_in elements -> q [rows][cols]
+ * codes with row stride ld_q bytes, scale [rows] fp32.  cols, ld_in and ld_q
+ * must be multiples of 8 and in, q 16-byte aligned. */
+int h3_quantize_rows_e4m3(const h3_bf16* in, int64_t ld_in, int rows, int cols, h3_e4m3* q, int64_t ld_q,
+                          float* scale, void* stream);
+
+/* A3 / A8 with e4m3 output: the fp32 values h3_adaln_norm_modulate would
+ * round to bf16 are row-quantised instead.  xq [L_pad][D] codes, xs [L_pad]
+ * fp32 (padding rows: codes 0, scale 0). */
+int h3_adaln_norm_modulate_e4m3(const h3_dims* dims, const h3_ranges* ranges, const float* x, const float* mod,
+                                int branch, h3_e4m3* xq, float* xs, void* stream);
+
+/* A4 + A5 from e4m3 operands: as h3_qkv_qknorm_mrope with xm = (xq, xs)
+ * [L_pad][D] and Wqkv = (Wq, Ws) [3I][D], Ws per output channel.  q, k, v
+ * bf16 head-major [H][L_pad][128]. */
+int h3_qkv_qknorm_mrope_e4m3(const h3_dims* dims, const h3_ranges* ranges, const h3_e4m3* xq, const float* xs,
+                             const h3_e4m3* Wq, const float* Ws, const h3_bf16* qn_w, const h3_bf16* kn_w,
+                             const float* pos, int flags, h3_bf16* q, h3_bf16* k, h3_bf16* v, void* stream);
+
+/* A7 from e4m3 operands: as h3_gated_residual with o = (oq, os) [L_pad][I]
+ * (e.g. the attention output through h3_quantize_rows_e4m3) and
+ * Wo = (Wq, Ws) [D][I]. */
+int h3_gated_residual_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_e4m3* oq,
+                           const float* os, const h3_e4m3* Wq, const float* Ws, const float* mod, int branch,
+                           void* stream);
+
+/* Bytes of the h3_ffn_swiglu_e4m3 workspace: the bf16 hidden state
+ * [L_pad][F], its codes [L_pad][F] and their scales [L_pad] fp32. */
+size_t h3_ffn_e4m3_workspace_bytes(const h3_dims* dims, int L_pad);
+
+/* A9 from e4m3 operands: h = bf16(SiLU(xm Wg^T) (.) (xm Wu^T)) with
+ * xm = (xq, xs) and Wgu = (Wgu_q, Wgu_s) [2F][D] (gate rows then up rows),
+ * then h row-quantised, then x[r] += gate_mlp_m (.) (h Wd^T)[r] with
+ * Wd = (Wd_q, Wd_s) [D][F].  ws: caller-owned scratch of
+ * h3_ffn_e4m3_workspace_bytes() bytes, 256-byte aligned. */
+int h3_ffn_swiglu_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_e4m3* xq,
+                       const float* xs, const h3_e4m3* Wgu_q, const float* Wgu_s, const h3_e4m3* Wd_q,
+                       const float* Wd_s, const float* mod, void* ws, void* stream);
+
+/* Block weights (e4m3 codes with per-output-channel scales) and buffers for
+ * h3_block_forward_e4m3. */
+typedef struct h3_block_weights_e4m3 {
+  const h3_e4m3* Wqkv; const float* Wqkv_s; /* [3I][D], [3I] */
+  const h3_bf16* qn_w;                      /* [128] */
+  const h3_bf16* kn_w;                      /* [128] */
+  const h3_e4m3* Wo;   const float* Wo_s;   /* [D][I], [D] */
+  const h3_e4m3* Wgu;  const float* Wgu_s;  /* [2F][D], [2F] */
+  const h3_e4m3* Wd;   const float* Wd_s;   /* [D][F], [D] */
+} h3_block_weights_e4m3;
+
+typedef struct h3_block_buffers_e4m3 {
+  h3_e4m3* xq; float* xs; /* [L_pad][D], [L_pad] */
+  h3_bf16* q;             /* [H][L_pad][128] */
+  h3_bf16* k;
+  h3_bf16* v;
+  h3_bf16* o;             /* [L_pad][I] */
+  h3_e4m3* oq; float* os; /* [L_pad][I], [L_pad] */
+  void* ws;               /* h3_ffn_e4m3_workspace_bytes() */
+} h3_block_buffers_e4m3;
+
+/* One whole block with e4m3 GEMMs: h3_adaln_norm_modulate_e4m3 (MSA),
+ * h3_qkv_qknorm_mrope_e4m3, h3_attention (bf16), h3_quantize_rows_e4m3 of o,
+ * h3_gated_residual_e4m3, h3_adaln_norm_modulate_e4m3 (MLP),
+ * h3_ffn_swiglu_e4m3.  Nothing is launched if any argument is invalid. */
+int h3_block_forward_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod,
+                          const float* pos, const h3_block_weights_e4m3* w, const h3_block_buffers_e4m3* buf,
+                          int flags, void* stream);
 
 #ifdef __cplusplus
 }

@@ -97,16 +97,53 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return t;
 }
 
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < (LN_THREADS + 31) / 32; ++i) t = fmaxf(t, red[i]);
+  return t;
+}
+
+// Per-row e4m3 scaling (OFP8 e4m3, saturating round-to-nearest-even): for a
+// row with amax = max |y| > 0, rscale = 448 / amax and scale = amax / 448 (both
+// IEEE fp32 divisions), code = e4m3(y * rscale) with the product rounded to
+// fp32; a zero row has rscale = scale = 0.
+__device__ __forceinline__ void e4m3_row_scales(float amax, float& rscale, float& scale) {
+  rscale = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+  scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 0.f;
+}
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d, float rs) {
+  return cvt_e4m3x2(__fmul_rn(a, rs), __fmul_rn(b, rs)) | (cvt_e4m3x2(__fmul_rn(c, rs), __fmul_rn(d, rs)) << 16);
+}
+
+// E4M3 = false: out is bf16 [L_pad][D].  E4M3 = true: out is e4m3 codes
+// [L_pad][D] (bytes) with one fp32 scale per row in out_scale, quantised
+// from the fp32 values of the modulated row.
+template <bool E4M3>
 __global__ void __launch_bounds__(LN_THREADS) ln_modulate_kernel(const float* __restrict__ x,
                                                                   const float* __restrict__ mod, int branch,
                                                                   RangeArgs rg, int L, int D, float eps,
-                                                                  bf16* __restrict__ out) {
+                                                                  void* __restrict__ out,
+                                                                  float* __restrict__ out_scale) {
   __shared__ float red[(LN_THREADS + 31) / 32];
   const int row = blockIdx.x;
   const int nv = D / 4;
-  bf16* orow = out + (long)row * D;
+  bf16* orow = static_cast<bf16*>(out) + (long)row * D;
+  uint8_t* qrow = static_cast<uint8_t*>(out) + (long)row * D;
   if (row >= L) {
-    for (int i = threadIdx.x; i < nv; i += LN_THREADS) *reinterpret_cast<uint2*>(orow + 4 * i) = make_uint2(0, 0);
+    for (int i = threadIdx.x; i < nv; i += LN_THREADS) {
+      if (E4M3)
+        *reinterpret_cast<uint32_t*>(qrow + 4 * i) = 0u;
+      else
+        *reinterpret_cast<uint2*>(orow + 4 * i) = make_uint2(0, 0);
+    }
+    if (E4M3 && threadIdx.x == 0) out_scale[row] = 0.f;
     return;
   }
   const float4* xr = reinterpret_cast<const float4*>(x + (long)row * D);
@@ -135,6 +172,7 @@ __global__ void __launch_bounds__(LN_THREADS) ln_modulate_kernel(const float* __
   const int m = range_of(row, rg.start, rg.count);
   const float4* shift = mod ? reinterpret_cast<const float4*>(mod + (long)(m * 6 + 3 * branch + 0) * D) : nullptr;
   const float4* scale = mod ? reinterpret_cast<const float4*>(mod + (long)(m * 6 + 3 * branch + 1) * D) : nullptr;
+  float amax = 0.f;
 #pragma unroll
   for (int k = 0; k < LN_VPT; ++k) {
     const int i = threadIdx.x + k * LN_THREADS;
@@ -147,8 +185,56 @@ __global__ void __launch_bounds__(LN_THREADS) ln_modulate_kernel(const float* __
         c = fmaf(c, 1.f + sc.z, sh.z);
         d = fmaf(d, 1.f + sc.w, sh.w);
       }
-      *reinterpret_cast<uint2*>(orow + 4 * i) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+      if (E4M3) {
+        v[k] = make_float4(a, b, c, d);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d))));
+      } else {
+        *reinterpret_cast<uint2*>(orow + 4 * i) = make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+      }
     }
+  }
+  if (E4M3) {
+    float rs, sc;
+    e4m3_row_scales(block_max(amax, red), rs, sc);
+    if (threadIdx.x == 0) out_scale[row] = sc;
+#pragma unroll
+    for (int k = 0; k < LN_VPT; ++k) {
+      const int i = threadIdx.x + k * LN_THREADS;
+      if (i < nv) *reinterpret_cast<uint32_t*>(qrow + 4 * i) = e4m3x4(v[k].x, v[k].y, v[k].z, v[k].w, rs);
+    }
+  }
+}
+
+// ------------------------------------------------------------ row quantiser
+// One CTA per row of a bf16 matrix: amax over the row, then codes with the
+// row scaling above.  cols, ld_in and ld_q are multiples of 8.
+__global__ void __launch_bounds__(LN_THREADS) quantize_rows_e4m3_kernel(const bf16* __restrict__ in, long ld_in,
+                                                                         int cols, uint8_t* __restrict__ q,
+                                                                         long ld_q, float* __restrict__ scale) {
+  __shared__ float red[(LN_THREADS + 31) / 32];
+  const int row = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(in + (long)row * ld_in);
+  const int n8 = cols / 8;
+  float amax = 0.f;
+  for (int i = threadIdx.x; i < n8; i += LN_THREADS) {
+    const uint4 w = __ldg(src + i);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  float rs, sc;
+  e4m3_row_scales(block_max(amax, red), rs, sc);
+  if (threadIdx.x == 0) scale[row] = sc;
+  uint2* dst = reinterpret_cast<uint2*>(q + (long)row * ld_q);
+  for (int i = threadIdx.x; i < n8; i += LN_THREADS) {
+    const uint4 w = __ldg(src + i);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+    dst[i] = make_uint2(e4m3x4(f0.x, f0.y, f1.x, f1.y, rs), e4m3x4(f2.x, f2.y, f3.x, f3.y, rs));
   }
 }
 
@@ -263,7 +349,26 @@ cudaError_t launch_ln_modulate(const float* x, const float* mod, int branch, con
     rg.start[m] = rstart[m];
     rg.count[m] = rcount[m];
   }
-  ln_modulate_kernel<<<L_pad, LN_THREADS, 0, stream>>>(x, mod, branch, rg, L, D, eps, out);
+  ln_modulate_kernel<false><<<L_pad, LN_THREADS, 0, stream>>>(x, mod, branch, rg, L, D, eps, out, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_modulate_e4m3(const float* x, const float* mod, int branch, const int* rstart,
+                                    const int* rcount, int L, int L_pad, int D, float eps, uint8_t* out,
+                                    float* out_scale, cudaStream_t stream) {
+  RangeArgs rg;
+  for (int m = 0; m < 3; ++m) {
+    rg.start[m] = rstart[m];
+    rg.count[m] = rcount[m];
+  }
+  ln_modulate_kernel<true><<<L_pad, LN_THREADS, 0, stream>>>(x, mod, branch, rg, L, D, eps, out, out_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_rows_e4m3(const bf16* in, long ld_in, int rows, int cols, uint8_t* q, long ld_q,
+                                      float* scale, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  quantize_rows_e4m3_kernel<<<rows, LN_THREADS, 0, stream>>>(in, ld_in, cols, q, ld_q, scale);
   return cudaGetLastError();
 }
 

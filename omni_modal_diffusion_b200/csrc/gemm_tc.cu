@@ -53,6 +53,19 @@ __device__ __forceinline__ void ld_chunk(uint32_t taddr, float* v) {
   tmem_ld32(taddr, reinterpret_cast<uint32_t*>(v));
 }
 
+// e4m3 operands: the 32 accumulator columns of a chunk (B rows b0 .. b0 + 31)
+// times a_scale[m] * b_scale[b]; B rows past the end scale to 0.  No-op for
+// bf16 operands.
+__device__ __forceinline__ void scale_chunk(const GemmEpilogue& e, float* v, int m, int b0) {
+  if (e.a_scale == nullptr) return;
+  const float sa = (m < e.a_rows) ? e.a_scale[m] : 0.f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int b = b0 + j;
+    v[j] *= sa * (b < e.b_rows ? __ldg(e.b_scale + b) : 0.f);
+  }
+}
+
 // ------------------------------------------------------------ epilogues
 __device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb, int m, int n0) {
 #pragma unroll 1
@@ -62,6 +75,7 @@ __device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb
     float v[32];
     ld_chunk(tb + c * 32, v);
     tmem_wait_ld();
+    scale_chunk(e, v, m, nc);
     if (m < e.M) {
       float* dst = static_cast<float*>(e.out) + (long)(e.row_off + m) * e.ldo + nc;
       if (nc + 32 <= e.N) {
@@ -87,6 +101,7 @@ __device__ __forceinline__ void epi_gated_resid(const GemmEpilogue& e, uint32_t 
     float v[32];
     ld_chunk(tb + c * 32, v);
     tmem_wait_ld();
+    scale_chunk(e, v, m, nc);
     if (mod_id >= 0) {
       if (nc + 32 <= e.N) {
 #pragma unroll
@@ -116,6 +131,8 @@ __device__ __forceinline__ void epi_swiglu(const GemmEpilogue& e, uint32_t tb, i
     ld_chunk(tb + c * 32, g);
     ld_chunk(tb + 128 + c * 32, u);
     tmem_wait_ld();
+    scale_chunk(e, g, m, nt * 128 + c * 32);
+    scale_chunk(e, u, m, e.N + nt * 128 + c * 32);
     if (m < e.M) {
       uint32_t packed[16];
 #pragma unroll
@@ -130,6 +147,21 @@ __device__ __forceinline__ void epi_swiglu(const GemmEpilogue& e, uint32_t tb, i
             make_uint4(packed[j], packed[j + 1], packed[j + 2], packed[j + 3]);
     }
   }
+}
+
+// sin and cos of a RoPE angle on the MUFU unit.  The angle is first reduced
+// to [-pi, pi] with 2 pi split into its nearest fp32 value H = 6.28318548...
+// and the remainder T = 2 pi - H = -1.7484556e-7 (two-term Cody-Waite
+// reduction: r = (a - k H) - k T, each step one fused multiply-add), which
+// keeps |r - (a - 2 pi k)| within a few fp32 ulps of r for the angles here
+// (|a| < 10^4); __sincosf is then accurate to ~2^-21 on [-pi, pi].  The
+// library's accurate sincosf took twice as long over the whole QKV GEMM with
+// e4m3 operands (the epilogue, not the MMAs, bounded it).
+__device__ __forceinline__ void rope_sincos(float a, float* s, float* c) {
+  const float k = rintf(a * 0.159154937f);  // a / (2 pi)
+  float r = fmaf(-k, 6.28318548f, a);
+  r = fmaf(-k, -1.74845553e-7f, r);
+  __sincosf(r, s, c);
 }
 
 __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int m, int n0, const float* freq,
@@ -150,6 +182,8 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
 #pragma unroll
     for (int c = 0; c < 4; ++c) ld_chunk(tb + half * 128 + c * 32, v + c * 32);
     tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) scale_chunk(e, v + c * 32, m, n + c * 32);
     if (part < 2) {
       float ss = 0.f;
 #pragma unroll
@@ -168,7 +202,7 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
         const int ax = axis_of_pair[i];
         const float pa = ax == 0 ? p3[0] : (ax == 1 ? p3[1] : p3[2]);
         float s, c;
-        sincosf(pa * freq[i], &s, &c);
+        rope_sincos(pa * freq[i], &s, &c);
         const float a = v[2 * i], b = v[2 * i + 1];
         v[2 * i] = a * c - b * s;
         v[2 * i + 1] = a * s + b * c;
@@ -200,6 +234,7 @@ __device__ __forceinline__ void epi_unpatch(const GemmEpilogue& e, uint32_t tb, 
     float v[32];
     ld_chunk(tb + c * 32, v);
     tmem_wait_ld();
+    scale_chunk(e, v, m, nc);
     if (m < e.M) {
       for (int jj = 0; jj < 32 && nc + jj < e.N; ++jj) {
         const int f = nc + jj;
@@ -211,9 +246,13 @@ __device__ __forceinline__ void epi_unpatch(const GemmEpilogue& e, uint32_t tb, 
   }
 }
 
+// F8: e4m3 operands (kind::f8f6f4), a K step of 128 one-byte elements; else
+// bf16 (kind::f16), a K step of 64.  Both stage 128-byte rows.
+template <bool F8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmProblem p) {
+  constexpr int KSTEP = F8 ? 2 * BK : BK;  // elements per stage
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -268,7 +307,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int m_tiles = (p.M + BM - 1) / BM;
   const int num_tiles = m_tiles * p.n_tiles;
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int num_kb = (p.K + KSTEP - 1) / KSTEP;
   const bool swiglu = e.mode == EPI_SWIGLU;
 
   if (warp == 0) {
@@ -285,9 +324,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(smA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * BK, mt * BM);
-          tma_load_2d(smB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * BK, b0);
-          tma_load_2d(smB + stage * B_STAGE_BYTES + B_STAGE_BYTES / 2, &tmB, &full[stage], kb * BK, b1);
+          tma_load_2d(smA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * KSTEP, mt * BM);
+          tma_load_2d(smB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * KSTEP, b0);
+          tma_load_2d(smB + stage * B_STAGE_BYTES + B_STAGE_BYTES / 2, &tmB, &full[stage], kb * KSTEP, b1);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -296,7 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // The whole warp runs the issue loop, converged; one elected lane issues.
-    const uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+    const uint32_t idesc = F8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, BN, false);
     // descriptors computed once; per MMA only the start address moves
     // (16-byte units: a 32-byte K step is +2)
     const uint64_t a_desc0 = sdesc_sw128(smem_u32(smA), 16, 1024);
@@ -316,8 +355,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t ad = a_desc0 + (uint64_t)((stage * A_STAGE_BYTES) >> 4);
         const uint64_t bd = b_desc0 + (uint64_t)((stage * B_STAGE_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+        for (int kk = 0; kk < BK / 16; ++kk) {  // 4 MMAs of 32 bytes of K
+          if constexpr (F8)
+            umma_e4m3(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          else
+            umma_bf16(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
@@ -375,9 +418,11 @@ constexpr int P_B_BYTES = 128 * BK * 2;             // 16 KB (half of the 256 co
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 512;
 
+template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const GemmProblem p) {
+  constexpr int KSTEP = F8 ? 2 * BK : BK;  // elements per stage
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -434,7 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
   const int m_pairs = (p.M + 255) / 256;
   const int num_tiles = m_pairs * p.n_tiles;
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int num_kb = (p.K + KSTEP - 1) / KSTEP;
   const bool swiglu = e.mode == EPI_SWIGLU;
 
   if (warp == 0) {
@@ -453,8 +498,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
           const uint32_t fb = leader_full0 + stage * 8;
-          tma_load_2d_pair(smA + stage * P_A_BYTES, &tmA, fb, kb * BK, arow);
-          tma_load_2d_pair(smB + stage * P_B_BYTES, &tmB, fb, kb * BK, brow);
+          tma_load_2d_pair(smA + stage * P_A_BYTES, &tmA, fb, kb * KSTEP, arow);
+          tma_load_2d_pair(smB + stage * P_B_BYTES, &tmB, fb, kb * KSTEP, brow);
           ++issued;
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
@@ -466,7 +511,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (leader) {
       // The leader's whole warp runs the issue loop, converged; one elected lane issues.
-      const uint32_t idesc = idesc_bf16_f32(256, 256, false);
+      const uint32_t idesc = F8 ? idesc_e4m3_f32(256, 256) : idesc_bf16_f32(256, 256, false);
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(smA), 16, 1024);
       const uint64_t b_desc0 = sdesc_sw128(smem_u32(smB), 16, 1024);
       int stage = 0;
@@ -484,8 +529,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
           const uint64_t ad = a_desc0 + (uint64_t)((stage * P_A_BYTES) >> 4);
           const uint64_t bd = b_desc0 + (uint64_t)((stage * P_B_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {  // 4 MMAs of 32 bytes of K
+            if constexpr (F8)
+              umma_e4m3_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
+                             (kb | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16_pair(d_tmem, ad + (uint64_t)(kk * 2), bd + (uint64_t)(kk * 2), idesc,
+                             (kb | kk) != 0 ? 1u : 0u);
+          }
           umma_commit_pair(&empty[stage]);
           if (++stage == P_STAGES) { stage = 0; phase ^= 1; }
         }
@@ -553,19 +604,29 @@ EncodeTiledFn encode_fn() {
 }  // namespace gemm_detail
 using namespace gemm_detail;
 
-// 2-D bf16 tensor map with 64-element (128-byte) inner boxes and 128-byte
-// swizzle; out-of-range elements read as zero.
-bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
-                    uint32_t box_rows) {
+// 2-D tensor map with 128-byte inner boxes (64 bf16 or 128 one-byte
+// elements) and 128-byte swizzle; out-of-range elements read as zero.
+static bool make_tmap_128b(CUtensorMap* map, CUtensorMapDataType dt, uint32_t elem_bytes, const void* base,
+                           uint64_t rows, uint64_t cols, uint64_t row_stride_elems, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {cols, rows};
-  cuuint64_t gstride[1] = {row_stride_elems * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t gstride[1] = {row_stride_elems * elem_bytes};
+  cuuint32_t box[2] = {128 / elem_bytes, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(map, dt, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                    uint32_t box_rows) {
+  return make_tmap_128b(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, row_stride_elems, box_rows);
+}
+
+static bool make_tmap_e4m3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint64_t row_stride_elems, uint32_t box_rows) {
+  return make_tmap_128b(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, row_stride_elems, box_rows);
 }
 
 int num_sms() {
@@ -594,16 +655,24 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, unsigned long long* do
 
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
   if (p.M <= 0) return cudaSuccess;
-  static unsigned long long attr_done = 0;
-  cudaError_t aerr = ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel), gemm_detail::SMEM_BYTES, &attr_done);
+  const bool f8 = p.f8 != 0;
+  if (f8 && (p.a_scale == nullptr || p.b_scale == nullptr)) return cudaErrorInvalidValue;
+  static unsigned long long attr_done[2] = {0, 0};
+  const void* k1 = f8 ? reinterpret_cast<const void*>(gemm_tc_kernel<true>)
+                      : reinterpret_cast<const void*>(gemm_tc_kernel<false>);
+  cudaError_t aerr = ensure_smem_attr(k1, gemm_detail::SMEM_BYTES, &attr_done[f8 ? 1 : 0]);
   if (aerr != cudaSuccess) return aerr;
   CUtensorMap tmA, tmB;
-  if (!make_tmap_bf16(&tmA, p.A, (uint64_t)p.M, (uint64_t)p.K, (uint64_t)p.lda, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16(&tmB, p.B, (uint64_t)p.N_b_rows, (uint64_t)p.K, (uint64_t)p.ldb, 128))
-    return cudaErrorInvalidValue;
+  auto make = f8 ? make_tmap_e4m3 : make_tmap_bf16;
+  if (!make(&tmA, p.A, (uint64_t)p.M, (uint64_t)p.K, (uint64_t)p.lda, 128)) return cudaErrorInvalidValue;
+  if (!make(&tmB, p.B, (uint64_t)p.N_b_rows, (uint64_t)p.K, (uint64_t)p.ldb, 128)) return cudaErrorInvalidValue;
   const int m_tiles = (p.M + gemm_detail::BM - 1) / gemm_detail::BM;
   const int tiles = m_tiles * p.n_tiles;
   GemmProblem q = p;
+  q.epi.a_scale = f8 ? p.a_scale : nullptr;
+  q.epi.b_scale = f8 ? p.b_scale : nullptr;
+  q.epi.a_rows = p.M;
+  q.epi.b_rows = p.N_b_rows;
   if (q.group_m <= 0) {
     // A band of row tiles whose A panel (128 rows x K bf16 each) takes about
     // 24 MB of L2, so it stays resident while B streams past.  Measured on
@@ -613,7 +682,7 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
 #ifndef H3_GEMM_BAND_BYTES
 #define H3_GEMM_BAND_BYTES (24ll << 20)
 #endif
-    const long long panel = 128ll * p.K * 2;
+    const long long panel = 128ll * p.K * (f8 ? 1 : 2);
     long long g = H3_GEMM_BAND_BYTES / (panel > 0 ? panel : 1);
     q.group_m = (int)(g < 1 ? 1 : (g > m_tiles ? m_tiles : g));
   }
@@ -625,9 +694,10 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
   // QKV GEMM from 1.30 / 5.33 ms to 1.27 / 5.24 ms, but is up to 5% slower
   // on the FFN's gate/up and down GEMMs at 32,160 tokens, so callers choose.
   if (H3_GEMM_PAIR && p.pair == 1 && p.M > 128) {
-    static unsigned long long attr2_done = 0;
-    cudaError_t err2 = ensure_smem_attr(reinterpret_cast<const void*>(gemm_detail::gemm_tc2_kernel),
-                                        gemm_detail::P_SMEM_BYTES, &attr2_done);
+    static unsigned long long attr2_done[2] = {0, 0};
+    const void* k2 = f8 ? reinterpret_cast<const void*>(gemm_detail::gemm_tc2_kernel<true>)
+                        : reinterpret_cast<const void*>(gemm_detail::gemm_tc2_kernel<false>);
+    cudaError_t err2 = ensure_smem_attr(k2, gemm_detail::P_SMEM_BYTES, &attr2_done[f8 ? 1 : 0]);
     if (err2 != cudaSuccess) return err2;
     const int m_pairs = (p.M + 255) / 256;
     GemmProblem q2 = q;
@@ -636,12 +706,19 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     const int pair_tiles = m_pairs * p.n_tiles;
     const int max_pairs = num_sms() / 2;
     const int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
-    gemm_detail::gemm_tc2_kernel<<<2 * pairs, gemm_detail::NUM_THREADS, gemm_detail::P_SMEM_BYTES, stream>>>(
-        tmA, tmB, q2);
+    if (f8)
+      gemm_detail::gemm_tc2_kernel<true><<<2 * pairs, gemm_detail::NUM_THREADS, gemm_detail::P_SMEM_BYTES, stream>>>(
+          tmA, tmB, q2);
+    else
+      gemm_detail::gemm_tc2_kernel<false><<<2 * pairs, gemm_detail::NUM_THREADS, gemm_detail::P_SMEM_BYTES,
+                                            stream>>>(tmA, tmB, q2);
     return cudaGetLastError();
   }
   const int grid = tiles < num_sms() ? tiles : num_sms();
-  gemm_tc_kernel<<<grid, gemm_detail::NUM_THREADS, gemm_detail::SMEM_BYTES, stream>>>(tmA, tmB, q);
+  if (f8)
+    gemm_tc_kernel<true><<<grid, gemm_detail::NUM_THREADS, gemm_detail::SMEM_BYTES, stream>>>(tmA, tmB, q);
+  else
+    gemm_tc_kernel<false><<<grid, gemm_detail::NUM_THREADS, gemm_detail::SMEM_BYTES, stream>>>(tmA, tmB, q);
   return cudaGetLastError();
 }
 

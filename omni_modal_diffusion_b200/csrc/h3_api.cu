@@ -108,6 +108,65 @@ void set_ranges(GemmEpilogue& e, const h3_ranges* r) {
   }
 }
 
+// The block's GEMM problems, shared by the bf16 and e4m3 entry points (the
+// e4m3 ones then set f8 and the scales).
+GemmProblem qkv_problem(const h3_dims* dims, const h3_ranges* ranges, const void* xm, const void* Wqkv,
+                        const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, h3_bf16* q, h3_bf16* k,
+                        h3_bf16* v) {
+  const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
+  GemmProblem p = gemm_base(xm, D, Lp, D, Wqkv, D, 3 * I, (3 * I + 255) / 256);
+  p.pair = 1;
+  GemmEpilogue& ep = p.epi;
+  ep.mode = EPI_QKV;
+  ep.M = Lp;
+  ep.N = 3 * I;
+  set_ranges(ep, ranges);
+  ep.q = reinterpret_cast<bf16*>(q);
+  ep.k = reinterpret_cast<bf16*>(k);
+  ep.v = reinterpret_cast<bf16*>(v);
+  ep.qn_w = reinterpret_cast<const bf16*>(qn_w);
+  ep.kn_w = reinterpret_cast<const bf16*>(kn_w);
+  ep.pos = pos;
+  ep.L_pad = Lp;
+  ep.I = I;
+  ep.rope_t = dims->rope_t;
+  ep.rope_h = dims->rope_h;
+  ep.rope_w = dims->rope_w;
+  ep.theta = dims->theta;
+  ep.eps_qk = dims->eps_qk;
+  return p;
+}
+
+// x += gate[slot] * (A W^T), A [L_pad][K], W [D][K]
+GemmProblem gated_problem(const h3_dims* dims, const h3_ranges* ranges, float* x, const void* A, int K,
+                          const void* W, const float* mod, int gate_slot) {
+  const int D = dims->D, Lp = ranges->L_pad;
+  GemmProblem p = gemm_base(A, K, Lp, K, W, K, D, (D + 255) / 256);
+  p.epi.mode = EPI_GATED_RESID;
+  p.epi.M = Lp;
+  p.epi.N = D;
+  p.epi.ldo = D;
+  p.epi.out = x;
+  set_ranges(p.epi, ranges);
+  p.epi.mod = mod;
+  p.epi.gate_slot = gate_slot;
+  p.epi.D = D;
+  return p;
+}
+
+// ws = bf16(SiLU(xm Wg^T) * (xm Wu^T)), Wgu = [gate rows; up rows]
+GemmProblem swiglu_problem(const h3_dims* dims, int Lp, const void* xm, const void* Wgu, void* ws) {
+  const int D = dims->D, F = dims->F;
+  GemmProblem p = gemm_base(xm, D, Lp, D, Wgu, D, 2 * F, F / 128);
+  p.b_second_half_off = F;
+  p.epi.mode = EPI_SWIGLU;
+  p.epi.M = Lp;
+  p.epi.N = F;
+  p.epi.ldo = F;
+  p.epi.out = ws;
+  return p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -222,27 +281,7 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
   H3_REQUIRE_PTR(q);
   H3_REQUIRE_PTR(k);
   H3_REQUIRE_PTR(v);
-  const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
-  GemmProblem p = gemm_base(xm, D, Lp, D, Wqkv, D, 3 * I, (3 * I + 255) / 256);
-  p.pair = 1;
-  GemmEpilogue& ep = p.epi;
-  ep.mode = EPI_QKV;
-  ep.M = Lp;
-  ep.N = 3 * I;
-  set_ranges(ep, ranges);
-  ep.q = reinterpret_cast<bf16*>(q);
-  ep.k = reinterpret_cast<bf16*>(k);
-  ep.v = reinterpret_cast<bf16*>(v);
-  ep.qn_w = reinterpret_cast<const bf16*>(qn_w);
-  ep.kn_w = reinterpret_cast<const bf16*>(kn_w);
-  ep.pos = pos;
-  ep.L_pad = Lp;
-  ep.I = I;
-  ep.rope_t = dims->rope_t;
-  ep.rope_h = dims->rope_h;
-  ep.rope_w = dims->rope_w;
-  ep.theta = dims->theta;
-  ep.eps_qk = dims->eps_qk;
+  GemmProblem p = qkv_problem(dims, ranges, xm, Wqkv, qn_w, kn_w, pos, q, k, v);
   cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_qkv_qknorm_mrope");
   return ok();
@@ -285,18 +324,8 @@ int h3_gated_residual(const h3_dims* dims, const h3_ranges* ranges, float* x, co
   H3_REQUIRE_PTR(o);
   H3_REQUIRE_PTR(Wo);
   H3_REQUIRE_PTR(mod);
-  const int D = dims->D, I = dims->I, Lp = ranges->L_pad;
-  GemmProblem p = gemm_base(o, I, Lp, I, Wo, I, D, (D + 255) / 256);
+  GemmProblem p = gated_problem(dims, ranges, x, o, dims->I, Wo, mod, 3 * branch + 2);
   p.pair = 1;
-  p.epi.mode = EPI_GATED_RESID;
-  p.epi.M = Lp;
-  p.epi.N = D;
-  p.epi.ldo = D;
-  p.epi.out = x;
-  set_ranges(p.epi, ranges);
-  p.epi.mod = mod;
-  p.epi.gate_slot = 3 * branch + 2;
-  p.epi.D = D;
   cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_gated_residual");
   return ok();
@@ -317,27 +346,12 @@ int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const 
   H3_REQUIRE_PTR(Wd);
   H3_REQUIRE_PTR(mod);
   H3_REQUIRE_PTR(ws);
-  const int D = dims->D, F = dims->F, Lp = ranges->L_pad;
+  const int Lp = ranges->L_pad;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  GemmProblem p1 = gemm_base(xm, D, Lp, D, Wgu, D, 2 * F, F / 128);
-  p1.b_second_half_off = F;
-  p1.epi.mode = EPI_SWIGLU;
-  p1.epi.M = Lp;
-  p1.epi.N = F;
-  p1.epi.ldo = F;
-  p1.epi.out = ws;
+  GemmProblem p1 = swiglu_problem(dims, Lp, xm, Wgu, ws);
   cudaError_t e = launch_gemm(p1, st);
   if (e != cudaSuccess) return cuda_fail(e, "h3_ffn_swiglu: gate/up");
-  GemmProblem p2 = gemm_base(ws, F, Lp, F, Wd, F, D, (D + 255) / 256);
-  p2.epi.mode = EPI_GATED_RESID;
-  p2.epi.M = Lp;
-  p2.epi.N = D;
-  p2.epi.ldo = D;
-  p2.epi.out = x;
-  set_ranges(p2.epi, ranges);
-  p2.epi.mod = mod;
-  p2.epi.gate_slot = 5;
-  p2.epi.D = D;
+  GemmProblem p2 = gated_problem(dims, ranges, x, ws, dims->F, Wd, mod, 5);
   e = launch_gemm(p2, st);
   if (e != cudaSuccess) return cuda_fail(e, "h3_ffn_swiglu: down");
   return ok();
@@ -491,4 +505,5 @@ int h3_set_wait_limit_ns(uint64_t ns) {
 }  // extern "C"
 
 // Workspace-free variant of h3_ffn_swiglu (uses this file's checks and launcher).
+#include "h3_fp8.cu"
 #include "h3_noalloc.cu"

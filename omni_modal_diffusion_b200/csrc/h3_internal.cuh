@@ -41,6 +41,12 @@ struct GemmEpilogue {
   float theta, eps_qk;
   // EPI_UNPATCH: token grid (T, Ht, Wt), latent channels
   int Ht, Wt, C_lat;
+  // e4m3 operands: acc[m][n] *= a_scale[m] * b_scale[n] before the epilogue
+  // (a_scale per A row, b_scale per B row); null for bf16 operands.  Set by
+  // launch_gemm from GemmProblem.
+  const float* a_scale;
+  const float* b_scale;
+  int a_rows, b_rows;
 };
 
 struct GemmProblem {
@@ -54,6 +60,11 @@ struct GemmProblem {
   int group_m;    // tile order: bands of group_m row tiles sweep all column tiles (L2 reuse of A)
   int pair;       // 1: CTA-pair kernel (256 x 256 tiles over two SMs) when M > 128; 0: one CTA per tile
   int b_second_half_off;  // SwiGLU: row offset of the "up" half in B (= F); else 128
+  // e4m3 operands (kind::f8f6f4): A and B hold one-byte codes (lda / ldb in
+  // bytes), scaled per A row and per B row; 0 for bf16.
+  int f8;
+  const float* a_scale;
+  const float* b_scale;
   GemmEpilogue epi;
 };
 
@@ -77,6 +88,11 @@ cudaError_t launch_pack(const bf16* video, int T, int Hl, int Wl, int C_lat, int
                         uint8_t* mod_ids, float* x, int D, cudaStream_t stream);
 cudaError_t launch_ln_modulate(const float* x, const float* mod, int branch, const int* rstart, const int* rcount,
                                int L, int L_pad, int D, float eps, bf16* out, cudaStream_t stream);
+cudaError_t launch_ln_modulate_e4m3(const float* x, const float* mod, int branch, const int* rstart,
+                                    const int* rcount, int L, int L_pad, int D, float eps, uint8_t* out,
+                                    float* out_scale, cudaStream_t stream);
+cudaError_t launch_quantize_rows_e4m3(const bf16* in, long ld_in, int rows, int cols, uint8_t* q, long ld_q,
+                                      float* scale, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
 cudaError_t launch_exp2_fma_pipe(const float* x, float* y, long long n, cudaStream_t stream);
 cudaError_t launch_euler_bf16(float* lat, const float* vel, long long n, float dsigma, bf16* out,

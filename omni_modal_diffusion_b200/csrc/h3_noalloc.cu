@@ -59,7 +59,7 @@ extern "C" int h3_ffn_swiglu_noalloc(const h3_dims* dims, const h3_ranges* range
   H3_REQUIRE_PTR(Wgu);
   H3_REQUIRE_PTR(Wd);
   H3_REQUIRE_PTR(mod);
-  const int D = dims->D, F = dims->F, Lp = ranges->L_pad;
+  const int F = dims->F, Lp = ranges->L_pad;
   const size_t need = (size_t)Lp * (size_t)F * 2;
   if (need > kStaticWsBytes)
     return fail(H3_ERR_SHAPE,
@@ -71,25 +71,10 @@ extern "C" int h3_ffn_swiglu_noalloc(const h3_dims* dims, const h3_ranges* range
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // gate/up GEMM writes every element [0, L_pad) x [0, F) of the workspace
   // that the down GEMM then reads, so nothing in it needs to start at zero.
-  GemmProblem p1 = gemm_base(xm, D, Lp, D, Wgu, D, 2 * F, F / 128);
-  p1.b_second_half_off = F;
-  p1.epi.mode = EPI_SWIGLU;
-  p1.epi.M = Lp;
-  p1.epi.N = F;
-  p1.epi.ldo = F;
-  p1.epi.out = ws;
+  GemmProblem p1 = swiglu_problem(dims, Lp, xm, Wgu, ws);
   cudaError_t e = launch_gemm(p1, st);
   if (e != cudaSuccess) return cuda_fail(e, "h3_ffn_swiglu_noalloc: gate/up");
-  GemmProblem p2 = gemm_base(ws, F, Lp, F, Wd, F, D, (D + 255) / 256);
-  p2.epi.mode = EPI_GATED_RESID;
-  p2.epi.M = Lp;
-  p2.epi.N = D;
-  p2.epi.ldo = D;
-  p2.epi.out = x;
-  set_ranges(p2.epi, ranges);
-  p2.epi.mod = mod;
-  p2.epi.gate_slot = 5;
-  p2.epi.D = D;
+  GemmProblem p2 = gated_problem(dims, ranges, x, ws, F, Wd, mod, 5);
   e = launch_gemm(p2, st);
   if (e != cudaSuccess) return cuda_fail(e, "h3_ffn_swiglu_noalloc: down");
   return ok();

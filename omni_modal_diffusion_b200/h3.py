@@ -26,6 +26,8 @@ EXPORTS = (
     "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
     "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_exp2_fma_pipe", "h3_block_forward",
     "h3_euler_step_bf16", "h3_selftest_wait_timeout",
+    "h3_quantize_rows_e4m3", "h3_adaln_norm_modulate_e4m3", "h3_qkv_qknorm_mrope_e4m3", "h3_gated_residual_e4m3",
+    "h3_ffn_e4m3_workspace_bytes", "h3_ffn_swiglu_e4m3", "h3_block_forward_e4m3",
 )
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
 
@@ -55,6 +57,18 @@ class BlockWeights(ctypes.Structure):
 
 class BlockBuffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("xm", "q", "k", "v", "o", "ws")]
+
+
+E4M3_WEIGHT_FIELDS = ("Wqkv", "Wqkv_s", "qn_w", "kn_w", "Wo", "Wo_s", "Wgu", "Wgu_s", "Wd", "Wd_s")
+E4M3_BUFFER_FIELDS = ("xq", "xs", "q", "k", "v", "o", "oq", "os", "ws")
+
+
+class BlockWeightsE4m3(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in E4M3_WEIGHT_FIELDS]
+
+
+class BlockBuffersE4m3(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in E4M3_BUFFER_FIELDS]
 
 
 _lib = None
@@ -91,6 +105,14 @@ def lib() -> ctypes.CDLL:
             "h3_device_status": (ci, [vp, ctypes.POINTER(ci)]),
             "h3_set_wait_limit_ns": (ci, [ctypes.c_uint64]),
             "h3_selftest_wait_timeout": (ci, [ctypes.c_uint64, vp]),
+            "h3_quantize_rows_e4m3": (ci, [vp, ctypes.c_int64, ci, ci, vp, ctypes.c_int64, vp, vp]),
+            "h3_adaln_norm_modulate_e4m3": (ci, [pd, pr, vp, vp, ci, vp, vp, vp]),
+            "h3_qkv_qknorm_mrope_e4m3": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp]),
+            "h3_gated_residual_e4m3": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, ci, vp]),
+            "h3_ffn_e4m3_workspace_bytes": (ctypes.c_size_t, [pd, ci]),
+            "h3_ffn_swiglu_e4m3": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
+            "h3_block_forward_e4m3": (ci, [pd, pr, vp, vp, vp, ctypes.POINTER(BlockWeightsE4m3),
+                                           ctypes.POINTER(BlockBuffersE4m3), ci, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -250,3 +272,66 @@ def h3_selftest_wait_timeout(limit_ns: int, stream=None):
 
 def h3_set_wait_limit_ns(ns: int):
     _check(lib().h3_set_wait_limit_ns(ns))
+
+
+# ------------------------------------------------------------ e4m3 (FP8) GEMMs
+# Codes are uint8 tensors, scales float32 (one per row / output channel).
+
+def h3_quantize_rows_e4m3(x, q, scale, stream=None):
+    """Row-quantise a 2-D bf16 tensor into e4m3 codes q (uint8, same shape) and
+    per-row scales (float32 [rows])."""
+    if x.dim() != 2 or q.shape != x.shape or scale.numel() != x.shape[0]:
+        raise ValueError("x [rows, cols], q [rows, cols] and scale [rows] required")
+    _check(lib().h3_quantize_rows_e4m3(_ptr(x, BF16, "x"), x.shape[1], x.shape[0], x.shape[1], _ptr(q, U8, "q"),
+                                       q.shape[1], _ptr(scale, F32, "scale"), _stream(stream)))
+
+
+def h3_adaln_norm_modulate_e4m3(dims, ranges, x, mod, branch, xq, xs, stream=None):
+    _check(lib().h3_adaln_norm_modulate_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                                             _ptr(mod, F32, "mod"), branch, _ptr(xq, U8, "xq"), _ptr(xs, F32, "xs"),
+                                             _stream(stream)))
+
+
+def h3_qkv_qknorm_mrope_e4m3(dims, ranges, xq, xs, Wq, Ws, qn_w, kn_w, pos, q, k, v, flags=H3_QK_NORM_ROPE_IN_QKV,
+                             stream=None):
+    _check(lib().h3_qkv_qknorm_mrope_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(xq, U8, "xq"),
+                                          _ptr(xs, F32, "xs"), _ptr(Wq, U8, "Wq"), _ptr(Ws, F32, "Ws"),
+                                          _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"), _ptr(pos, F32, "pos"),
+                                          flags, _ptr(q, BF16, "q"), _ptr(k, BF16, "k"), _ptr(v, BF16, "v"),
+                                          _stream(stream)))
+
+
+def h3_gated_residual_e4m3(dims, ranges, x, oq, os_, Wq, Ws, mod, branch=H3_MSA, stream=None):
+    _check(lib().h3_gated_residual_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                                        _ptr(oq, U8, "oq"), _ptr(os_, F32, "os"), _ptr(Wq, U8, "Wq"),
+                                        _ptr(Ws, F32, "Ws"), _ptr(mod, F32, "mod"), branch, _stream(stream)))
+
+
+def h3_ffn_e4m3_workspace_bytes(dims, L_pad: int) -> int:
+    return int(lib().h3_ffn_e4m3_workspace_bytes(ctypes.byref(dims), L_pad))
+
+
+def h3_ffn_swiglu_e4m3(dims, ranges, x, xq, xs, Wgu_q, Wgu_s, Wd_q, Wd_s, mod, ws, stream=None):
+    _check(lib().h3_ffn_swiglu_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"), _ptr(xq, U8, "xq"),
+                                    _ptr(xs, F32, "xs"), _ptr(Wgu_q, U8, "Wgu_q"), _ptr(Wgu_s, F32, "Wgu_s"),
+                                    _ptr(Wd_q, U8, "Wd_q"), _ptr(Wd_s, F32, "Wd_s"), _ptr(mod, F32, "mod"),
+                                    _ptr(ws, U8, "ws"), _stream(stream)))
+
+
+def block_weights_e4m3(W: dict) -> BlockWeightsE4m3:
+    """Pointer struct of one block's e4m3 weights: codes (uint8) and scales
+    (float32) under the names of E4M3_WEIGHT_FIELDS; qn_w, kn_w bf16."""
+    dt = {"qn_w": BF16, "kn_w": BF16}
+    return BlockWeightsE4m3(*(_ptr(W[n], dt.get(n, F32 if n.endswith("_s") else U8), n) for n in E4M3_WEIGHT_FIELDS))
+
+
+def block_buffers_e4m3(B: dict) -> BlockBuffersE4m3:
+    dt = {"xq": U8, "xs": F32, "q": BF16, "k": BF16, "v": BF16, "o": BF16, "oq": U8, "os": F32, "ws": U8}
+    return BlockBuffersE4m3(*(_ptr(B[n], dt[n], n) for n in E4M3_BUFFER_FIELDS))
+
+
+def h3_block_forward_e4m3(dims, ranges, x, mod, pos, weights: BlockWeightsE4m3, buffers: BlockBuffersE4m3,
+                          flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_block_forward_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                                       _ptr(mod, F32, "mod"), _ptr(pos, F32, "pos"), ctypes.byref(weights),
+                                       ctypes.byref(buffers), flags, _stream(stream)))

@@ -77,6 +77,45 @@ class H3BlockStep:
         h3.h3_adaln_norm_modulate(d, r, self.x, mod, h3.H3_MLP, self.xm, stream=stream)
         h3.h3_ffn_swiglu(d, r, self.x, self.xm, W["Wgu"], W["Wd"], mod, self.ws, stream=stream)
 
+    # ---------------------------------------------------------- e4m3 GEMMs
+    def quantize_block_weights_e4m3(self, W=None, stream=None) -> dict:
+        """e4m3 codes + per-output-channel scales of a block's GEMM weights
+        (h3_quantize_rows_e4m3 on the GPU), with qn_w / kn_w passed through."""
+        W = W or self.W
+        out = {"qn_w": W["qn_w"], "kn_w": W["kn_w"]}
+        for n in ("Wqkv", "Wo", "Wgu", "Wd"):
+            t = W[n]
+            q = torch.empty(t.shape, dtype=torch.uint8, device=self.device)
+            sc = torch.empty(t.shape[0], dtype=torch.float32, device=self.device)
+            h3.h3_quantize_rows_e4m3(t, q, sc, stream=stream)
+            out[n], out[n + "_s"] = q, sc
+        return out
+
+    def alloc_e4m3(self):
+        """Activation buffers of the e4m3 path (codes and row scales)."""
+        Lp, D, I = self.ranges.L_pad, self.w.D, self.w.I
+        dev = self.device
+        self.xq = torch.empty(Lp, D, dtype=torch.uint8, device=dev)
+        self.xs = torch.empty(Lp, dtype=torch.float32, device=dev)
+        self.oq = torch.empty(Lp, I, dtype=torch.uint8, device=dev)
+        self.os = torch.empty(Lp, dtype=torch.float32, device=dev)
+        self.ws8 = torch.empty(h3.h3_ffn_e4m3_workspace_bytes(self.dims, Lp), dtype=torch.uint8, device=dev)
+
+    def block_e4m3(self, mod, W8: dict, stream=None):
+        """One block over self.x with the four GEMMs in e4m3 (W8 from
+        quantize_block_weights_e4m3; alloc_e4m3 called once before)."""
+        d, r = self.dims, self.ranges
+        h3.h3_adaln_norm_modulate_e4m3(d, r, self.x, mod, h3.H3_MSA, self.xq, self.xs, stream=stream)
+        h3.h3_qkv_qknorm_mrope_e4m3(d, r, self.xq, self.xs, W8["Wqkv"], W8["Wqkv_s"], W8["qn_w"], W8["kn_w"],
+                                    self.pos, self.q, self.k, self.v, stream=stream)
+        h3.h3_attention(d, r, self.q, self.k, self.v, self.o, stream=stream)
+        h3.h3_quantize_rows_e4m3(self.o, self.oq, self.os, stream=stream)
+        h3.h3_gated_residual_e4m3(d, r, self.x, self.oq, self.os, W8["Wo"], W8["Wo_s"], mod, h3.H3_MSA,
+                                  stream=stream)
+        h3.h3_adaln_norm_modulate_e4m3(d, r, self.x, mod, h3.H3_MLP, self.xq, self.xs, stream=stream)
+        h3.h3_ffn_swiglu_e4m3(d, r, self.x, self.xq, self.xs, W8["Wgu"], W8["Wgu_s"], W8["Wd"], W8["Wd_s"], mod,
+                              self.ws8, stream=stream)
+
     def head(self, stream=None):
         w = self.w
         h3.h3_head_unpack(self.dims, self.ranges, self.x, self.W["W_vhead"], self.W["W_ahead"],
@@ -96,10 +135,11 @@ class H3BlockStep:
         self.euler(lat_video, lat_audio, sig_video, sig_audio, stream)
 
     # kernels launched by one step (for the launch count the bench reports)
-    def launches_per_step(self) -> int:
+    def launches_per_step(self, e4m3: bool = False) -> int:
         r = self.ranges
         embed = (1 if r.count[2] > 0 else 0) + 1 + (1 if r.L_pad > r.L else 0) + sum(1 for c in r.count if c > 0)
-        block = 1 + 1 + 1 + 1 + 1 + 2
+        # LN, QKV, attention, [quantise o,] out-projection, LN, FFN (2 GEMMs [+ quantise h])
+        block = 1 + 1 + 1 + 1 + 1 + 2 + (2 if e4m3 else 0)
         head = 1 + (1 if r.count[2] > 0 else 0) + (1 if r.count[1] > 0 else 0)
         return embed + block + head + 2
 
