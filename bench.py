@@ -69,8 +69,11 @@ def bytes_per_call(w, L, Lp):
 # kernel changes (see profiles/).
 TRAFFIC = {
     # mean over the block's QKV, out-projection, FFN gate/up and FFN down
-    # launches (6.203 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel"): 1.551e9,
+    # launches (6.580 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel"): 1.645e9,
+    # the same four launches with e4m3 operands (2.580 GB / 4),
+    # profiles/gemm_tc_kernel_e4m3_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.645e9,
     # profiles/attention_tc_kernel_768sq_2s.md
     ("768sq_2s", "attention_tc_kernel"): 0.4355e9,
 }
@@ -426,9 +429,11 @@ def run_e4m3(args, w):
                    "quantisation": "OFP8 e4m3, per-token activation and per-output-channel weight scales"},
         "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel<e4m3>", "achieved": round(gemm_tf, 1),
                      "peak": round(peak_f8, 1), "unit": "TFLOP/s", "frac": round(gemm_tf / peak_f8, 4),
-                     "peak_kind": "2 x bf16 sustained of measured (nominal e4m3 / bf16 ratio)", "traffic": None},
+                     "peak_kind": "2 x bf16 sustained of measured (nominal e4m3 / bf16 ratio)",
+                     "traffic": TRAFFIC.get((w.name, "gemm_tc_kernel<e4m3>"))},
         "kernels": {"gemm_tc_kernel<e4m3>": {"ms_per_step": round(gemm_ms, 4), "tflops": round(gemm_tf, 1),
-                                             "frac": round(gemm_tf / peak_f8, 4)},
+                                             "frac": round(gemm_tf / peak_f8, 4), "launches_per_step": 4,
+                                             "traffic_per_launch": TRAFFIC.get((w.name, "gemm_tc_kernel<e4m3>"))},
                     "attention_tc_kernel": {"ms_per_step": round(per_call["h3_attention"], 4),
                                             "tflops": round(fl["h3_attention"] / (per_call["h3_attention"] / 1e3)
                                                             / 1e12, 1)}},

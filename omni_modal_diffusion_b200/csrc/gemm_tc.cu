@@ -59,10 +59,22 @@ __device__ __forceinline__ void ld_chunk(uint32_t taddr, float* v) {
 __device__ __forceinline__ void scale_chunk(const GemmEpilogue& e, float* v, int m, int b0) {
   if (e.a_scale == nullptr) return;
   const float sa = (m < e.a_rows) ? e.a_scale[m] : 0.f;
+  if (b0 + 32 <= e.b_rows) {  // b0 is a multiple of 32 and b_scale 16-byte aligned
+    const float4* bs = reinterpret_cast<const float4*>(e.b_scale + b0);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int b = b0 + j;
-    v[j] *= sa * (b < e.b_rows ? __ldg(e.b_scale + b) : 0.f);
+    for (int j = 0; j < 32; j += 4) {
+      const float4 b = __ldg(bs + j / 4);
+      v[j] *= sa * b.x;
+      v[j + 1] *= sa * b.y;
+      v[j + 2] *= sa * b.z;
+      v[j + 3] *= sa * b.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int b = b0 + j;
+      v[j] *= sa * (b < e.b_rows ? __ldg(e.b_scale + b) : 0.f);
+    }
   }
 }
 
