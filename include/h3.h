@@ -74,8 +74,9 @@ typedef struct h3_dims {
 } h3_dims;
 
 /* Packed-sequence ranges: rows [start[m], start[m] + count[m]) hold modality
- * m; the three ranges tile [0, L) without overlap; L_pad = L rounded up to a
- * multiple of 128 ([shouss] §2.2). */
+ * m; the three ranges tile [0, L) without overlap ([shouss] §2.2); L_pad is
+ * a multiple of 128 with L <= L_pad (h3_make_ranges gives L rounded up; a
+ * sequence-parallel shard, h3_sp_make_layout, may pad further). */
 typedef struct h3_ranges {
   int start[3];
   int count[3];
@@ -351,6 +352,71 @@ typedef struct h3_block_buffers_e4m3 {
 int h3_block_forward_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod,
                           const float* pos, const h3_block_weights_e4m3* w, const h3_block_buffers_e4m3* buf,
                           int flags, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sequence parallelism (Ulysses), the pages' own multi-GPU deployment of the
+ * trunk ([gojay] §7.2: Ulysses degree 4).  N ranks (N <= H3_SP_MAX_RANKS,
+ * H % N == 0) each hold a contiguous shard of L_shard rows of the packed
+ * sequence: rank r owns global rows [r L_shard, (r + 1) L_shard) of a
+ * sequence padded to L_total = N L_shard.  Everything token-local (LN +
+ * modulation, the GEMMs, the FFN, the residual) runs on the shard with the
+ * shard's h3_ranges.  Attention needs every token of a head, so the QKV
+ * call writes head group g (heads [g H/N, (g + 1) H/N)) of its shard
+ * straight into rank g's q/k/v buffers (an all-to-all fused into the GEMM
+ * epilogue), and the attention call writes each output row straight into
+ * the o buffer of the row's owner (the second all-to-all, fused into the
+ * attention epilogue).  Peer buffers are device pointers the caller maps
+ * (CUDA IPC or symmetric memory between GPUs; plain local buffers when the
+ * ranks share one GPU).  Between the QKV calls of all ranks and any
+ * attention call, and between the attention calls and the out-projections,
+ * every rank's writes must be complete and visible: the caller orders them
+ * (a barrier on the streams, e.g. a collective or event wait). */
+#define H3_SP_MAX_RANKS 8
+
+typedef struct h3_sp_layout {
+  int n_ranks;   /* N */
+  int rank;      /* this rank */
+  int L;         /* valid tokens of the whole sequence */
+  int L_shard;   /* rows per shard, a multiple of 128: ceil(L / N / 128) * 128 */
+  int L_total;   /* N * L_shard */
+  int row0;      /* rank * L_shard: first global row of this shard */
+  int heads;     /* H / N: heads per rank after the exchange */
+} h3_sp_layout;
+
+/* Host only.  The layout of rank `rank` of n_ranks for the global ranges,
+ * and the shard's own ranges (modality ranges intersected with the shard,
+ * relative to its first row; shard->L = its valid rows, shard->L_pad =
+ * L_shard).  Every shard must hold at least one valid row:
+ * L > (n_ranks - 1) * L_shard, else H3_ERR_SHAPE. */
+int h3_sp_make_layout(const h3_dims* dims, const h3_ranges* global, int n_ranks, int rank, h3_sp_layout* out,
+                      h3_ranges* shard);
+
+/* Device pointers of every rank's exchange buffers (index = rank):
+ *   q[g], k[g], v[g]: rank g's [H/N][L_total][128] bf16 (head-major; global
+ *                     row order, so the attention of rank g sees the whole
+ *                     sequence for its heads)
+ *   o[g]:             rank g's [L_shard][H * 128] bf16 attention output */
+typedef struct h3_sp_peers {
+  h3_bf16* q[H3_SP_MAX_RANKS];
+  h3_bf16* k[H3_SP_MAX_RANKS];
+  h3_bf16* v[H3_SP_MAX_RANKS];
+  h3_bf16* o[H3_SP_MAX_RANKS];
+} h3_sp_peers;
+
+/* A4 + A5 on this rank's shard (xm [L_shard][D], pos [L_shard][3]) with the
+ * q, k, v of head h written to rank h / (H/N), local head h % (H/N), global
+ * row row0 + m: the QKV GEMM and the first all-to-all in one kernel. */
+int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3_sp_layout* layout,
+                           const h3_bf16* xm, const h3_bf16* Wqkv, const h3_bf16* qn_w, const h3_bf16* kn_w,
+                           const float* pos, int flags, const h3_sp_peers* peers, void* stream);
+
+/* A6 for this rank's H/N heads over all L tokens (its q, k, v =
+ * peers->q/k/v[rank], filled by every rank's h3_qkv_qknorm_mrope_sp), with
+ * output row R (global) written to peers->o[R / L_shard], row R % L_shard,
+ * columns of head (rank H/N + h): attention and the second all-to-all in
+ * one kernel.  Rows >= L are written as 0. */
+int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers, int flags,
+                    void* stream);
 
 #ifdef __cplusplus
 }

@@ -62,10 +62,20 @@ constexpr int POLY_EVERY = H3_ATTN_POLY_EVERY;
 #endif
 constexpr bool SPLIT_P = H3_ATTN_SPLIT_P != 0;
 
+// Where output rows go: row R (of the L_pad rows this launch covers) to
+// shard[R / L_shard], row R % L_shard, row stride ld, head column offset
+// (head0 + h) * 128.  One shard for a plain launch; one per rank (the owners
+// of the rows) for a sequence-parallel one.
+struct AttnOut {
+  long ld;
+  int head0, L_shard;
+  bf16* shard[8];
+};
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ out, int H, int L, int L_pad,
-                        float scale_log2) {
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnOut out, int H, int L,
+                        int L_pad, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -310,7 +320,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int grow = qt * TILE + r;
       const float inv = (grow < L) ? 1.0f / l_sum : 0.0f;
-      bf16* dst = out + (long)grow * (H * 128) + h * 128;
+      const int owner = grow / out.L_shard;
+      bf16* dst = out.shard[owner] + (long)(grow - owner * out.L_shard) * out.ld + (out.head0 + h) * 128;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         float o[32];
@@ -354,9 +365,23 @@ cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
   if (!make_tmap_bf16(&tk, p.k, rows, 128, 128, 128)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tv, p.v, rows, 128, 128, 128)) return cudaErrorInvalidValue;
   const int n_qt = p.L_pad / attn_detail::TILE;
+  AttnOut out;
+  memset(&out, 0, sizeof(out));
+  if (p.sp_n > 0) {
+    if (p.sp_n > 8 || p.sp_L_shard <= 0 || (long)p.sp_n * p.sp_L_shard < p.L_pad) return cudaErrorInvalidValue;
+    out.ld = p.sp_ld;
+    out.head0 = p.sp_head0;
+    out.L_shard = p.sp_L_shard;
+    for (int i = 0; i < p.sp_n; ++i) out.shard[i] = p.sp_o[i];
+  } else {
+    out.ld = (long)p.H * 128;
+    out.head0 = 0;
+    out.L_shard = p.L_pad;
+    out.shard[0] = p.o;
+  }
   dim3 grid((n_qt + 1) / 2, p.H);
   attention_tc_kernel<<<grid, attn_detail::NUM_THREADS, attn_detail::SMEM_BYTES, stream>>>(
-      tq, tk, tv, p.o, p.H, p.L, p.L_pad, p.scale_log2);
+      tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2);
   return cudaGetLastError();
 }
 

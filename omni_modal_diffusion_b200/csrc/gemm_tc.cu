@@ -221,8 +221,15 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
       }
     }
     if (m < e.M) {
-      bf16* base = part == 0 ? e.q : (part == 1 ? e.k : e.v);
-      bf16* dst = base + ((long)h * e.L_pad + m) * 128;
+      bf16* dst;
+      if (e.sp_n > 0) {  // sequence parallel: straight into the head group's rank
+        const int g = h / e.sp_heads, hl = h - g * e.sp_heads;
+        bf16* base = part == 0 ? e.sp_q[g] : (part == 1 ? e.sp_k[g] : e.sp_v[g]);
+        dst = base + ((long)hl * e.sp_L_total + e.sp_row0 + m) * 128;
+      } else {
+        bf16* base = part == 0 ? e.q : (part == 1 ? e.k : e.v);
+        dst = base + ((long)h * e.L_pad + m) * 128;
+      }
 #pragma unroll
       for (int d = 0; d < 128; d += 8) {
         uint4 o;
@@ -263,7 +270,7 @@ __device__ __forceinline__ void epi_unpatch(const GemmEpilogue& e, uint32_t tb, 
 template <bool F8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmProblem p) {
+                   const __grid_constant__ GemmProblem p) {
   constexpr int KSTEP = F8 ? 2 * BK : BK;  // elements per stage
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -433,7 +440,7 @@ constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 512;
 template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmProblem p) {
+                    const __grid_constant__ GemmProblem p) {
   constexpr int KSTEP = F8 ? 2 * BK : BK;  // elements per stage
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);

@@ -63,8 +63,8 @@ int check_dims(const h3_dims* d, const char* fn) {
 int check_ranges(const h3_ranges* r, const char* fn) {
   if (!r) return fail(H3_ERR_NULL, "%s: ranges is NULL", fn);
   if (r->L <= 0) return fail(H3_ERR_SHAPE, "%s: L must be positive (got %d)", fn, r->L);
-  if (r->L_pad % 128 != 0 || r->L_pad < r->L || r->L_pad - r->L >= 128)
-    return fail(H3_ERR_SHAPE, "%s: L_pad (%d) must be L (%d) rounded up to a multiple of 128", fn, r->L_pad, r->L);
+  if (r->L_pad % 128 != 0 || r->L_pad < r->L)
+    return fail(H3_ERR_SHAPE, "%s: L_pad (%d) must be a multiple of 128 and at least L (%d)", fn, r->L_pad, r->L);
   long total = 0;
   for (int m = 0; m < 3; ++m) {
     if (r->start[m] < 0 || r->count[m] < 0 || (long)r->start[m] + r->count[m] > r->L)
@@ -302,6 +302,7 @@ int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q,
   H3_REQUIRE_PTR(v);
   H3_REQUIRE_PTR(o);
   AttnProblem p;
+  memset(&p, 0, sizeof(p));
   p.q = reinterpret_cast<const bf16*>(q);
   p.k = reinterpret_cast<const bf16*>(k);
   p.v = reinterpret_cast<const bf16*>(v);
@@ -506,4 +507,5 @@ int h3_set_wait_limit_ns(uint64_t ns) {
 
 // Workspace-free variant of h3_ffn_swiglu (uses this file's checks and launcher).
 #include "h3_fp8.cu"
+#include "h3_sp.cu"
 #include "h3_noalloc.cu"

@@ -47,6 +47,13 @@ struct GemmEpilogue {
   const float* a_scale;
   const float* b_scale;
   int a_rows, b_rows;
+  // EPI_QKV, sequence parallel (sp_n > 0): head h of GEMM row m goes to rank
+  // h / sp_heads, local head h % sp_heads, row sp_row0 + m of its
+  // [sp_heads][sp_L_total][128] buffers sp_q / sp_k / sp_v.
+  int sp_n, sp_heads, sp_L_total, sp_row0;
+  bf16* sp_q[8];
+  bf16* sp_k[8];
+  bf16* sp_v[8];
 };
 
 struct GemmProblem {
@@ -79,6 +86,12 @@ struct AttnProblem {
   bf16* o;
   int H, L, L_pad;
   float scale_log2;  // log2(e) / sqrt(head_dim)
+  // Sequence parallel (sp_n > 0): o row R goes to sp_o[R / sp_L_shard], row
+  // R % sp_L_shard, row stride sp_ld elements, head column offset
+  // (sp_head0 + h) * 128; o is unused.
+  int sp_n, sp_L_shard, sp_head0;
+  long sp_ld;
+  bf16* sp_o[8];
 };
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream);
 

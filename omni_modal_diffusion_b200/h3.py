@@ -28,7 +28,9 @@ EXPORTS = (
     "h3_euler_step_bf16", "h3_selftest_wait_timeout",
     "h3_quantize_rows_e4m3", "h3_adaln_norm_modulate_e4m3", "h3_qkv_qknorm_mrope_e4m3", "h3_gated_residual_e4m3",
     "h3_ffn_e4m3_workspace_bytes", "h3_ffn_swiglu_e4m3", "h3_block_forward_e4m3",
+    "h3_sp_make_layout", "h3_qkv_qknorm_mrope_sp", "h3_attention_sp",
 )
+H3_SP_MAX_RANKS = 8
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
 
 
@@ -61,6 +63,14 @@ class BlockBuffers(ctypes.Structure):
 
 E4M3_WEIGHT_FIELDS = ("Wqkv", "Wqkv_s", "qn_w", "kn_w", "Wo", "Wo_s", "Wgu", "Wgu_s", "Wd", "Wd_s")
 E4M3_BUFFER_FIELDS = ("xq", "xs", "q", "k", "v", "o", "oq", "os", "ws")
+
+
+class SPLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("n_ranks", "rank", "L", "L_shard", "L_total", "row0", "heads")]
+
+
+class SPPeers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p * 8) for n in ("q", "k", "v", "o")]
 
 
 class BlockWeightsE4m3(ctypes.Structure):
@@ -113,6 +123,10 @@ def lib() -> ctypes.CDLL:
             "h3_ffn_swiglu_e4m3": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
             "h3_block_forward_e4m3": (ci, [pd, pr, vp, vp, vp, ctypes.POINTER(BlockWeightsE4m3),
                                            ctypes.POINTER(BlockBuffersE4m3), ci, vp]),
+            "h3_sp_make_layout": (ci, [pd, pr, ci, ci, ctypes.POINTER(SPLayout), pr]),
+            "h3_qkv_qknorm_mrope_sp": (ci, [pd, pr, ctypes.POINTER(SPLayout), vp, vp, vp, vp, vp, ci,
+                                            ctypes.POINTER(SPPeers), vp]),
+            "h3_attention_sp": (ci, [pd, ctypes.POINTER(SPLayout), ctypes.POINTER(SPPeers), ci, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -335,3 +349,41 @@ def h3_block_forward_e4m3(dims, ranges, x, mod, pos, weights: BlockWeightsE4m3, 
     _check(lib().h3_block_forward_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
                                        _ptr(mod, F32, "mod"), _ptr(pos, F32, "pos"), ctypes.byref(weights),
                                        ctypes.byref(buffers), flags, _stream(stream)))
+
+
+# ------------------------------------------------------------ sequence parallelism (Ulysses)
+
+def h3_sp_make_layout(dims, global_ranges, n_ranks: int, rank: int):
+    """(SPLayout, shard Ranges) of rank `rank` of n_ranks (host only)."""
+    lay, shard = SPLayout(), Ranges()
+    _check(lib().h3_sp_make_layout(ctypes.byref(dims), ctypes.byref(global_ranges), n_ranks, rank,
+                                   ctypes.byref(lay), ctypes.byref(shard)))
+    return lay, shard
+
+
+def sp_peers(q=None, k=None, v=None, o=None) -> SPPeers:
+    """Peer table from per-rank lists of CUDA tensors (index = rank); a list
+    may be None when the call does not use it."""
+    p = SPPeers()
+    for name, ts in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if ts is None:
+            continue
+        if len(ts) > H3_SP_MAX_RANKS:
+            raise ValueError(f"at most {H3_SP_MAX_RANKS} ranks")
+        arr = getattr(p, name)
+        for i, t in enumerate(ts):
+            arr[i] = _ptr(t, BF16, f"{name}[{i}]").value
+    return p
+
+
+def h3_qkv_qknorm_mrope_sp(dims, shard, layout, xm, Wqkv, qn_w, kn_w, pos, peers: SPPeers,
+                           flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_qkv_qknorm_mrope_sp(ctypes.byref(dims), ctypes.byref(shard), ctypes.byref(layout),
+                                        _ptr(xm, BF16, "xm"), _ptr(Wqkv, BF16, "Wqkv"), _ptr(qn_w, BF16, "qn_w"),
+                                        _ptr(kn_w, BF16, "kn_w"), _ptr(pos, F32, "pos"), flags, ctypes.byref(peers),
+                                        _stream(stream)))
+
+
+def h3_attention_sp(dims, layout, peers: SPPeers, flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_attention_sp(ctypes.byref(dims), ctypes.byref(layout), ctypes.byref(peers), flags,
+                                 _stream(stream)))
