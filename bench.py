@@ -462,7 +462,8 @@ def run_sampler(args, w):
     blocks = [{"Wqkv": rnd(3 * w.I, w.D, std=0.02), "qn_w": rnd(128, std=0.1) + 1, "kn_w": rnd(128, std=0.1) + 1,
                "Wo": rnd(w.D, w.I, std=0.02), "Wgu": rnd(2 * w.F, w.D, std=0.02), "Wd": rnd(w.D, w.F, std=0.02)}
               for _ in range(args.layers)]
-    smp = H3Sampler(w, io, blocks, device=dev)
+    weights_gb = sum(t.numel() * 2 for b_ in blocks for t in b_.values()) / 1e9
+    smp = H3Sampler(w, io, blocks, device=dev, e4m3=args.e4m3)
     L = smp.st.ranges.L
     n_total = args.warmup + args.steps
     text = rnd(w.n_text, w.D_text)
@@ -489,12 +490,13 @@ def run_sampler(args, w):
     assert h3.h3_device_status() == 0
     ms = a.elapsed_time(b) / args.steps
     fl = block_flops(w, L) * args.layers
-    return {"metric": "end-to-end denoise steps/s (layered flow sampler, bf16, 1xB200)",
+    kind = "e4m3 GEMMs, bf16 attention" if args.e4m3 else "bf16"
+    return {"metric": f"end-to-end denoise steps/s (layered flow sampler, {kind}, 1xB200)",
             "value": round(1e3 / ms, 4), "unit": "denoise steps/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init bf16 weights, N(0,1) latents)",
+            "vs_baseline": None, "dtype": kind, "data": "synthetic (random-init bf16 weights, N(0,1) latents)",
             "config": {"workload": w.name, "packed_tokens": L, "layers": args.layers,
-                       "weights_gb": round(sum(t.numel() * 2 for b_ in blocks for t in b_.values()) / 1e9, 1)},
+                       "weights_gb_bf16": round(weights_gb, 1)},
             "tokens_per_s_per_block": round(L * args.layers / (ms / 1e3), 1),
             "tflops": round(fl / (ms / 1e3) / 1e12, 1), "frac_of_bf16_sustained": round(
                 fl / (ms / 1e3) / 1e12 / _peaks()["bf16_tflops_sustained"], 4),

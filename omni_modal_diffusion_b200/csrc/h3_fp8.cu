@@ -129,7 +129,7 @@ int h3_ffn_swiglu_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, c
   H3_REQUIRE_PTR(Wd_s);
   H3_REQUIRE_PTR(mod);
   H3_REQUIRE_PTR(ws);
-  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(H3_ERR_SHAPE, "%s: ws must be 256-byte aligned", __func__);
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(H3_ERR_ALIGN, "%s: ws must be 256-byte aligned", __func__);
   const int F = dims->F, Lp = ranges->L_pad;
   const FfnE4m3Ws lay = ffn_e4m3_layout(Lp, F);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -180,7 +180,7 @@ int h3_block_forward_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x
   H3_REQUIRE_PTR(buf->v);
   H3_REQUIRE_PTR(buf->ws);
   if (reinterpret_cast<uintptr_t>(buf->ws) & 255u)
-    return fail(H3_ERR_SHAPE, "%s: ws must be 256-byte aligned", __func__);
+    return fail(H3_ERR_ALIGN, "%s: ws must be 256-byte aligned", __func__);
   const int I = dims->I, Lp = ranges->L_pad;
   H3_CHECK(h3_adaln_norm_modulate_e4m3(dims, ranges, x, mod, H3_MSA, buf->xq, buf->xs, stream));
   H3_CHECK(h3_qkv_qknorm_mrope_e4m3(dims, ranges, buf->xq, buf->xs, w->Wqkv, w->Wqkv_s, w->qn_w, w->kn_w, pos,

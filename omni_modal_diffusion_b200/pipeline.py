@@ -152,15 +152,31 @@ class H3Sampler:
     Per denoise step: pack + project the bf16 latents, n_layers blocks
     (h3_block_forward, modulation [step][layer][3][6][D]), head, then one
     Euler step per modality that also writes the bf16 latent for the next
-    step.  Orchestration only: every step runs in the library's kernels."""
+    step.  Orchestration only: every step runs in the library's kernels.
+
+    e4m3=True runs the blocks with their four GEMMs on e4m3 operands
+    (h3_block_forward_e4m3): each block's weights are quantised once on the
+    GPU here and the bf16 block weights are released."""
 
     def __init__(self, w: Workload, io_weights: dict, block_weights: list, device="cuda",
-                 shift_video: float = 12.0, shift_audio: float = 3.0):
+                 shift_video: float = 12.0, shift_audio: float = 3.0, e4m3: bool = False):
         self.st = H3BlockStep(w, device=device, weights=io_weights)
-        self.block_tensors = block_weights            # keep the tensors alive
-        self.blocks = [h3.block_weights(Wb) for Wb in block_weights]
         st = self.st
-        self.bufs = h3.block_buffers(st.xm, st.q, st.k, st.v, st.o, st.ws)
+        self.e4m3 = e4m3
+        if e4m3:
+            st.alloc_e4m3()
+            self.block_tensors = []
+            for i in range(len(block_weights)):
+                self.block_tensors.append(st.quantize_block_weights_e4m3(block_weights[i]))
+                block_weights[i] = None                # drop the bf16 copy as soon as it is quantised
+            torch.cuda.synchronize(st.device)
+            self.blocks = [h3.block_weights_e4m3(Wb) for Wb in self.block_tensors]
+            self.bufs = h3.block_buffers_e4m3({"xq": st.xq, "xs": st.xs, "q": st.q, "k": st.k, "v": st.v,
+                                               "o": st.o, "oq": st.oq, "os": st.os, "ws": st.ws8})
+        else:
+            self.block_tensors = block_weights            # keep the tensors alive
+            self.blocks = [h3.block_weights(Wb) for Wb in block_weights]
+            self.bufs = h3.block_buffers(st.xm, st.q, st.k, st.v, st.o, st.ws)
         self.shifts = (shift_video, shift_audio)
 
     @property
@@ -170,9 +186,9 @@ class H3Sampler:
     def step(self, s, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, sv, sa, stream=None):
         st = self.st
         st.embed(text, video_bf16, audio_bf16, stream)
+        forward = h3.h3_block_forward_e4m3 if self.e4m3 else h3.h3_block_forward
         for b in range(self.n_layers):
-            h3.h3_block_forward(st.dims, st.ranges, st.x, mod_all[s, b], st.pos, self.blocks[b], self.bufs,
-                                stream=stream)
+            forward(st.dims, st.ranges, st.x, mod_all[s, b], st.pos, self.blocks[b], self.bufs, stream=stream)
         st.head(stream)
         h3.h3_euler_step_bf16(lat_video, st.v_video, sv[s], sv[s + 1], video_bf16, stream=stream)
         h3.h3_euler_step_bf16(lat_audio, st.v_audio, sa[s], sa[s + 1], audio_bf16, stream=stream)
@@ -187,4 +203,5 @@ class H3Sampler:
 
     def launches_per_step(self) -> int:
         st = self.st
-        return st.launches_per_step() - 2 - 7 + 7 * self.n_layers + 2
+        per_block = 9 if self.e4m3 else 7
+        return st.launches_per_step() - 2 - 7 + per_block * self.n_layers + 2
