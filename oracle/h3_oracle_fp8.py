@@ -98,19 +98,25 @@ def quantize_rows(x) -> tuple[np.ndarray, np.ndarray]:
     """Per-row e4m3 quantisation of a 2-D array (values taken as fp32).
 
     Returns (codes uint8 [M, K], scale float32 [M]) with
-    dec(codes[r]) * scale[r] ~= x[r]."""
+    dec(codes[r]) * scale[r] ~= x[r].  Rows are processed in blocks only to
+    bound memory; every row follows the definition above on its own."""
     x32 = np.asarray(x, dtype=np.float32)
     M = x32.shape[0]
     codes = np.zeros(x32.shape, dtype=np.uint8)
     scale = np.zeros(M, dtype=np.float32)
-    for r in range(M):
-        amax = np.float32(np.max(np.abs(x32[r]))) if x32.shape[1] else np.float32(0)
-        if amax == 0:
-            continue  # zero row: scale 0, codes 0
-        rscale = np.float32(E4M3_MAX) / amax
-        scale[r] = amax / np.float32(E4M3_MAX)
-        y = (x32[r] * rscale).astype(np.float32)
-        codes[r] = e4m3_encode(y)
+    if x32.size == 0:
+        return codes, scale
+    for r0 in range(0, M, 1024):
+        blk = x32[r0:r0 + 1024]
+        amax = np.max(np.abs(blk), axis=1).astype(np.float32)
+        nz = amax > 0
+        safe = np.where(nz, amax, np.float32(1)).astype(np.float32)
+        rscale = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(0)).astype(np.float32)
+        scale[r0:r0 + len(blk)] = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(0))
+        y = (blk * rscale[:, None]).astype(np.float32)
+        c = e4m3_encode(y)
+        c[~nz] = 0  # zero row: scale 0, codes 0
+        codes[r0:r0 + len(blk)] = c
     return codes, scale
 
 

@@ -259,3 +259,51 @@ def test_block_e4m3_against_oracle(w):
     # separate the e4m3 block from the bf16 one.
     check_close(g - x0, ref - x0, "e4m3 block delta", max_rel_rms=0.35, mean_rel=2.5e-2)
     assert np.all(to_np(xg)[L:] == 0)
+
+
+def test_full_size_e4m3_qkv_and_ffn_sampled_rows():
+    """The e4m3 QKV (pair kernel, RMSNorm + RoPE epilogue) and FFN at the
+    full model widths (D 5376, 56 heads, F 14336) on the 768x768 2 s packing,
+    with 24 sampled rows carrying seeded activations (the other rows zero):
+    weights quantised per output channel by the oracle's quantiser, the
+    oracle evaluating the sampled rows only."""
+    from parity_util import oracle_ranges_and_pos as orp
+    w = S.WORKLOADS["768sq_2s"]
+    inp = S.make_inputs(w)
+    r, pos = orp(w)
+    L, Lp = r["L"], r["L_pad"]
+    rng = np.random.default_rng(5376)
+    rows = np.sort(rng.choice(L, 24, replace=False))
+    rows[0], rows[-1] = 0, L - 1
+    rows = np.unique(rows)
+    xm = np.zeros((Lp, w.D), np.float32)
+    xm[rows] = S.bf16_round(rng.standard_normal((len(rows), w.D), dtype=np.float32))
+    xq, xs = F8.quantize_rows(xm)
+    Wq, Ws = F8.quantize_weight(inp["Wqkv"])
+    d, rg = _dims(w, r)
+    pos_pad = np.zeros((Lp, 3), np.float32)
+    pos_pad[:L] = pos
+    q, k, v = (torch.empty(w.H, Lp, 128, dtype=torch.bfloat16, device=DEV) for _ in range(3))
+    h3.h3_qkv_qknorm_mrope_e4m3(d, rg, _u8(xq), _f32(xs), _u8(Wq), _f32(Ws), to_dev_bf16(inp["qn_w"], DEV),
+                                to_dev_bf16(inp["kn_w"], DEV), _f32(pos_pad), q, k, v)
+    ref = F8.qkv_qknorm_mrope_e4m3(xq[rows], xs[rows], Wq, Ws, inp["qn_w"], inp["kn_w"], pos[rows], w.H)
+    ridx = torch.from_numpy(rows).to(DEV)
+    for name, g, o in zip("qkv", (q, k, v), ref):
+        check_close(to_np(g[:, ridx, :]).transpose(1, 0, 2), o, f"e4m3 {name} rows", 3e-2, 3e-3)
+    del Wq, Ws
+    # FFN on the same rows
+    Wgu_q, Wgu_s = F8.quantize_weight(inp["Wgu"])
+    Wd_q, Wd_s = F8.quantize_weight(inp["Wd"])
+    x = np.zeros((Lp, w.D), np.float32)
+    x[:L] = rng.standard_normal((L, w.D), dtype=np.float32)
+    xg = _f32(x)
+    ws = torch.empty(h3.h3_ffn_e4m3_workspace_bytes(d, Lp), dtype=torch.uint8, device=DEV)
+    h3.h3_ffn_swiglu_e4m3(d, rg, xg, _u8(xq), _f32(xs), _u8(Wgu_q), _f32(Wgu_s), _u8(Wd_q), _f32(Wd_s),
+                          _f32(inp["mod"]), ws)
+    h = F8.swiglu_hidden_e4m3(xq[rows], xs[rows], Wgu_q, Wgu_s)
+    hq, hs = F8.quantize_rows(O.round_to_bf16(h))
+    ref = F8.ffn_down_e4m3(x[rows], hq, hs, Wd_q, Wd_s, inp["mod"], r, rows)
+    g = to_np(xg)[rows]
+    check_close(g - x[rows], ref - x[rows], "e4m3 ffn delta rows")
+    others = np.setdiff1d(np.arange(L), rows)[:64]
+    assert np.array_equal(to_np(xg)[others], x[others].astype(np.float64))   # zero rows: no change

@@ -30,9 +30,15 @@ def _built():
     torch.cuda.init()
 
 
-@pytest.mark.parametrize("n_ranks", [2, 3])
-def test_sp_block_matches_single_gpu_block_and_oracle(n_ranks):
-    w = RAGGED
+import dataclasses
+
+# 2,015 tokens (text 37, audio 58, video 5 x 16 x 24) and 8 heads: long enough
+# for four shards of 512 rows, the last one holding 479 valid rows
+LONG = dataclasses.replace(RAGGED, name="long", index=11, H=8, T_lat=5, H_lat=32, W_lat=48)
+
+
+@pytest.mark.parametrize("w,n_ranks", [(RAGGED, 2), (RAGGED, 3), (LONG, 4)], ids=["ragged2", "ragged3", "long4"])
+def test_sp_block_matches_single_gpu_block_and_oracle(w, n_ranks):
     inp = S.make_inputs(w)
     st = H3BlockStep(w, weights=inp)
     text, video, audio = (to_dev_bf16(inp[k], st.device) for k in ("text", "video", "audio"))
