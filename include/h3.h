@@ -243,6 +243,20 @@ typedef struct h3_block_buffers {
 int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod, const float* pos,
                      const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream);
 
+/* NEXT-3, a reading: the text refiner ("MiniMax-H3: native joint audio-video
+ * generation" (note.shouss.top) §3.2 config table: 2 text refiner blocks that
+ * prepare the text before the trunk; their structure is not stated).  Here
+ * a refiner block has the trunk block's form (h3_block_forward) and runs over
+ * the text range alone: the packed rows [0, count[TEXT]) of x (text comes
+ * first in the packing) as a text-only sequence, in place, each block with
+ * its own weights w[b] and modulation mods[b] ([3][6][D], only the text slot
+ * read); audio and video rows of x are read by nothing and left unchanged.
+ * pos: the packed positions (text rows are at (0, 0, 0)); buf: buffers for
+ * h3_block_forward at the packed L_pad (the text-only pass uses less).  No-op
+ * when there is no text or n_blocks == 0. */
+int h3_text_refine(const h3_dims* dims, const h3_ranges* ranges, float* x, int n_blocks, const float* const* mods,
+                   const float* pos, const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream);
+
 /* A11 for a sampler loop: h3_euler_step, and also writes the updated latent
  * rounded to bf16 into lat_bf16 (the transformer input of the next step). */
 int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, h3_bf16* lat_bf16,

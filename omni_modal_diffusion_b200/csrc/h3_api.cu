@@ -415,6 +415,31 @@ int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float si
   return ok();
 }
 
+int h3_text_refine(const h3_dims* dims, const h3_ranges* ranges, float* x, int n_blocks, const float* const* mods,
+                   const float* pos, const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream) {
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(ranges, __func__));
+  if (n_blocks < 0) return fail(H3_ERR_SHAPE, "%s: n_blocks must be >= 0", __func__);
+  const int n_text = ranges->count[H3_TEXT];
+  if (n_blocks == 0 || n_text == 0) return ok();
+  if (ranges->start[H3_TEXT] != 0)
+    return fail(H3_ERR_SHAPE, "%s: the text range must start at row 0 of the packing", __func__);
+  if (!mods || !w) return fail(H3_ERR_NULL, "%s: mods and w are required", __func__);
+  for (int b = 0; b < n_blocks; ++b)
+    if (!mods[b]) return fail(H3_ERR_NULL, "%s: mods[%d] is NULL", __func__, b);
+  h3_ranges t;
+  memset(&t, 0, sizeof(t));
+  t.start[H3_TEXT] = 0;
+  t.count[H3_TEXT] = n_text;
+  t.start[H3_AUDIO] = n_text;
+  t.start[H3_VIDEO] = n_text;
+  t.L = n_text;
+  t.L_pad = (n_text + 127) / 128 * 128;
+  for (int b = 0; b < n_blocks; ++b)
+    H3_CHECK(h3_block_forward(dims, &t, x, mods[b], pos, &w[b], buf, flags, stream));
+  return ok();
+}
+
 int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, h3_bf16* lat_bf16,
                        void* stream) {
   if (n < 0) return fail(H3_ERR_SHAPE, "h3_euler_step_bf16: n < 0");

@@ -28,7 +28,7 @@ EXPORTS = (
     "h3_euler_step_bf16", "h3_selftest_wait_timeout",
     "h3_quantize_rows_e4m3", "h3_adaln_norm_modulate_e4m3", "h3_qkv_qknorm_mrope_e4m3", "h3_gated_residual_e4m3",
     "h3_ffn_e4m3_workspace_bytes", "h3_ffn_swiglu_e4m3", "h3_block_forward_e4m3",
-    "h3_sp_make_layout", "h3_qkv_qknorm_mrope_sp", "h3_attention_sp",
+    "h3_sp_make_layout", "h3_qkv_qknorm_mrope_sp", "h3_attention_sp", "h3_text_refine",
 )
 H3_SP_MAX_RANKS = 8
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
@@ -127,6 +127,8 @@ def lib() -> ctypes.CDLL:
             "h3_qkv_qknorm_mrope_sp": (ci, [pd, pr, ctypes.POINTER(SPLayout), vp, vp, vp, vp, vp, ci,
                                             ctypes.POINTER(SPPeers), vp]),
             "h3_attention_sp": (ci, [pd, ctypes.POINTER(SPLayout), ctypes.POINTER(SPPeers), ci, vp]),
+            "h3_text_refine": (ci, [pd, pr, vp, ci, ctypes.POINTER(ctypes.c_void_p), vp,
+                                    ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockBuffers), ci, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -387,3 +389,17 @@ def h3_qkv_qknorm_mrope_sp(dims, shard, layout, xm, Wqkv, qn_w, kn_w, pos, peers
 def h3_attention_sp(dims, layout, peers: SPPeers, flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
     _check(lib().h3_attention_sp(ctypes.byref(dims), ctypes.byref(layout), ctypes.byref(peers), flags,
                                  _stream(stream)))
+
+
+def h3_text_refine(dims, ranges, x, mods: list, pos, weights: list, buffers: BlockBuffers,
+                   flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    """The text refiner blocks over the packed text rows of x, in place
+    (mods: per-block [3][6][D] float32 CUDA tensors; weights: per-block
+    BlockWeights)."""
+    n = len(weights)
+    if len(mods) != n:
+        raise ValueError("one modulation per refiner block")
+    mod_ptrs = (ctypes.c_void_p * max(n, 1))(*[_ptr(m, F32, "mod").value for m in mods])
+    w_arr = (BlockWeights * max(n, 1))(*weights)
+    _check(lib().h3_text_refine(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"), n, mod_ptrs,
+                                _ptr(pos, F32, "pos"), w_arr, ctypes.byref(buffers), flags, _stream(stream)))
