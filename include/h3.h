@@ -207,11 +207,11 @@ int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x,
  * [shouss] §5, §6).  lat, vel: fp32 device arrays of n elements. */
 int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream);
 
-/* Diagnostic: y[i] = 2^x[i] on the FMA pipe instead of the MUFU unit, the
- * form h3_attention can take for part of its softmax exponentials (a build
- * option, off by default): x clamped to >= -125, x = j + f with j = rint(x),
- * 2^f from a cubic (max relative error 7.5e-5 for x in [-125, 64]), 2^j added
- * to the exponent.  x, y: fp32 device arrays of n elements. */
+/* Diagnostic: y[i] = 2^x[i] on the FMA pipe instead of the MUFU unit (the
+ * form measured for part of attention's softmax exponentials, which took
+ * longer there): x clamped to >= -125, x = j + f with j = rint(x), 2^f from a
+ * cubic (max relative error 7.5e-5 for x in [-125, 64]), 2^j added to the
+ * exponent.  x, y: fp32 device arrays of n elements. */
 int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream);
 
 /* Block weights and scratch buffers for h3_block_forward (all device

@@ -36,19 +36,6 @@ constexpr int SMEM_BAR = SMEM_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
-// Tuning knobs (compile time): one pair in POLY_EVERY pairs of a full key
-// tile takes its exponentials on the FMA pipe (0 = none); SPLIT_P releases
-// P to the PV MMA in two halves instead of one.  Measured on B200 at 7,904
-// and 32,160 tokens: POLY_EVERY 0 / 8 / 4 / 2 -> 1.64 / 1.65 / 1.66-1.76 /
-// 1.70-1.78 ms and SPLIT_P 1 is 4-8% slower, because each softmax thread's
-// instruction latency, not MUFU throughput, bounds a phase in this layout.
-#ifndef H3_ATTN_POLY_EVERY
-#define H3_ATTN_POLY_EVERY 0
-#endif
-#ifndef H3_ATTN_SPLIT_P
-#define H3_ATTN_SPLIT_P 0
-#endif
-constexpr int POLY_EVERY = H3_ATTN_POLY_EVERY;
 // How the MMA issuer waits: polling (1) or suspending try_wait (0).  The
 // suspending wait leaves the issue slots of its sub-partition to the softmax
 // warps that share it: 1.486 vs 1.499 ms at 7,904 tokens, equal at 32,160.
@@ -60,7 +47,6 @@ constexpr int POLY_EVERY = H3_ATTN_POLY_EVERY;
 #else
 #define MMA_WAIT_WARP mbar_wait_warp
 #endif
-constexpr bool SPLIT_P = H3_ATTN_SPLIT_P != 0;
 
 // Where output rows go: row R (of the L_pad rows this launch covers) to
 // shard[R / L_shard], row R % L_shard, row stride ld, head column offset
@@ -90,9 +76,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* v_empty = bars + 7;   // [2] per V stage: freed after the tile's last PV MMA
   uint64_t* s_full = bars + 9;    // [2] per query tile
   uint64_t* o_final = bars + 11;  // [2] per query tile
-  uint64_t* p_full = bars + 13;   // [2 tiles][2 halves of the key tile]
-  uint64_t* drain = bars + 17;    // the MMA issuer's last commit before teardown
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* p_full = bars + 13;   // [2] per query tile: P in TMEM (4 warp arrivals)
+  uint64_t* drain = bars + 15;    // the MMA issuer's last commit before teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -110,8 +96,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[2 * s], 4);
-      mbar_init(&p_full[2 * s + 1], 4);
+      mbar_init(&p_full[s], 4);
       mbar_init(&o_final[s], 1);
     }
     mbar_init(drain, 1);
@@ -178,16 +163,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       umma_commit(&s_full[t]);
     };
-    // O_t += P_t V_j for keys [64 hf, 64 hf + 64), P_t (bf16, packed)
-    // read from TMEM where S_t was
-    auto issue_pv_half = [&](int t, int j, int hf) {
+    // O_t += P_t V_j, P_t (bf16, two per column) read from TMEM where S_t was
+    auto issue_pv = [&](int t, int j) {
       const uint64_t vd = v_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int kk = hf * 4 + k4;
+      for (int kk = 0; kk < 8; ++kk)
         umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
                          (j | kk) != 0 ? 1u : 0u);
-      }
     };
     bool ok = MMA_WAIT_WARP(q_full, 0) && MMA_WAIT_WARP(&k_full[0], 0);
     if (ok) {
@@ -199,15 +181,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int j = 0; j < nkv && ok; ++j) {
       const bool more = j + 1 < nkv;
       for (int t = 0; t < 2 && ok; ++t) {
-        for (int hf = 0; hf < 2; ++hf) {
-          if (SPLIT_P || hf == 0) {
-            if (!MMA_WAIT_WARP(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
-            if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-          }
-          issue_pv_half(t, j, hf);
-        }
-        if (!ok) break;
+        if (!MMA_WAIT_WARP(&p_full[t], j & 1)) { ok = false; break; }
+        if (t == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(t, j);
         if (more) {
           if (t == 0) {
             if (!MMA_WAIT_WARP(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
@@ -276,9 +253,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_st32(tO + c * 32, reinterpret_cast<const uint32_t*>(o));
         }
       }
-      // p = 2^(s * scale_log2 - m_ref); on full tiles some exponentials run
-      // on the FMA pipe (exp2_poly2) to relieve the MUFU unit; masked tiles
-      // use ex2 only so that masked keys give exactly 0.
+      // p = 2^(s * scale_log2 - m_ref) on the MUFU unit (masked keys, -inf,
+      // give exactly 0)
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
       const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
       uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -290,23 +266,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const int cc = hf * 64 + c;
-          float x0, x1, p0, p1;
+          float x0, x1;
           f2_unpack(f2_fma(f2_pack(s[cc], s[cc + 1]), sc2, nm2), x0, x1);
-          if (POLY_EVERY > 0 && full && ((c / 2) % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
-            exp2_poly2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_pack(p0, p1));
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tS + hf * 32, pk);
-        if (SPLIT_P || hf == 1) {
+        if (hf == 1) {
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[2 * t + (SPLIT_P ? hf : 0)]);
+          if (lane == 0) mbar_arrive(&p_full[t]);
         }
       }
       float a0, a1, a2, a3;
