@@ -69,11 +69,11 @@ def bytes_per_call(w, L, Lp):
 # kernel changes (see profiles/).
 TRAFFIC = {
     # mean over the block's QKV, out-projection, FFN gate/up and FFN down
-    # launches (6.096 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel"): 1.524e9,
-    # the same four launches with e4m3 operands (2.578 GB / 4),
+    # launches (6.089 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel"): 1.522e9,
+    # the same four launches with e4m3 operands (2.663 GB / 4),
     # profiles/gemm_tc_kernel_e4m3_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.6445e9,
+    ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.666e9,
     # profiles/attention_tc_kernel_768sq_2s.md
     ("768sq_2s", "attention_tc_kernel"): 0.4362e9,
 }

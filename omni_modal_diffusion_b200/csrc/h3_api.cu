@@ -142,6 +142,7 @@ GemmProblem gated_problem(const h3_dims* dims, const h3_ranges* ranges, float* x
                           const void* W, const float* mod, int gate_slot) {
   const int D = dims->D, Lp = ranges->L_pad;
   GemmProblem p = gemm_base(A, K, Lp, K, W, K, D, (D + 255) / 256);
+  p.pair = 1;
   p.epi.mode = EPI_GATED_RESID;
   p.epi.M = Lp;
   p.epi.N = D;
@@ -158,6 +159,7 @@ GemmProblem gated_problem(const h3_dims* dims, const h3_ranges* ranges, float* x
 GemmProblem swiglu_problem(const h3_dims* dims, int Lp, const void* xm, const void* Wgu, void* ws) {
   const int D = dims->D, F = dims->F;
   GemmProblem p = gemm_base(xm, D, Lp, D, Wgu, D, 2 * F, F / 128);
+  p.pair = 1;
   p.b_second_half_off = F;
   p.epi.mode = EPI_SWIGLU;
   p.epi.M = Lp;
@@ -326,7 +328,6 @@ int h3_gated_residual(const h3_dims* dims, const h3_ranges* ranges, float* x, co
   H3_REQUIRE_PTR(Wo);
   H3_REQUIRE_PTR(mod);
   GemmProblem p = gated_problem(dims, ranges, x, o, dims->I, Wo, mod, 3 * branch + 2);
-  p.pair = 1;
   cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_gated_residual");
   return ok();

@@ -104,7 +104,6 @@ int h3_gated_residual_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* 
   H3_REQUIRE_PTR(Ws);
   H3_REQUIRE_PTR(mod);
   GemmProblem p = with_e4m3(gated_problem(dims, ranges, x, oq, dims->I, Wq, mod, 3 * branch + 2), os, Ws);
-  p.pair = 1;
   cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_gated_residual_e4m3");
   return ok();
