@@ -7,6 +7,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/h3.h"
 #include "elementwise.cu"
 #include "gemm_tc.cu"
@@ -34,6 +36,15 @@ int ok() {
 int cuda_fail(cudaError_t e, const char* what) {
   return fail(H3_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
+
+// NVTX range over one C-ABI call, named after it, for a profiler that
+// attaches (NVTX3 is header-only: with no tool attached push and pop return
+// at once).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+#define H3_TRACE() NvtxRange h3_trace_range_(__func__)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -209,6 +220,7 @@ int h3_embed_pack(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* t
                   int audio_channels, int n_audio, int C_audio, const h3_bf16* W_text, const h3_bf16* W_vid,
                   const h3_bf16* W_aud, h3_bf16* patches, float* x_out, float* pos_out, uint8_t* mod_out,
                   void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   const int nt = ranges->count[H3_TEXT], na = ranges->count[H3_AUDIO], nv = ranges->count[H3_VIDEO];
@@ -256,6 +268,7 @@ int h3_embed_pack(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* t
 
 int h3_adaln_norm_modulate(const h3_dims* dims, const h3_ranges* ranges, const float* x, const float* mod,
                            int branch, h3_bf16* xm, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (branch != H3_MSA && branch != H3_MLP) return fail(H3_ERR_SHAPE, "%s: branch must be H3_MSA or H3_MLP", __func__);
@@ -271,6 +284,7 @@ int h3_adaln_norm_modulate(const h3_dims* dims, const h3_ranges* ranges, const f
 int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* xm, const h3_bf16* Wqkv,
                         const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags, h3_bf16* q,
                         h3_bf16* k, h3_bf16* v, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
@@ -292,6 +306,7 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
 int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q, const h3_bf16* k,
                  const h3_bf16* v, const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
                  h3_bf16* o, void* stream) {
+  H3_TRACE();
   (void)qn_w;
   (void)kn_w;
   (void)pos;
@@ -320,6 +335,7 @@ int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q,
 
 int h3_gated_residual(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* o,
                       const h3_bf16* Wo, const float* mod, int branch, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (branch != H3_MSA && branch != H3_MLP) return fail(H3_ERR_SHAPE, "%s: branch must be H3_MSA or H3_MLP", __func__);
@@ -340,6 +356,7 @@ size_t h3_ffn_workspace_bytes(const h3_dims* dims, int L_pad) {
 
 int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* xm,
                   const h3_bf16* Wgu, const h3_bf16* Wd, const float* mod, h3_bf16* ws, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   H3_REQUIRE_PTR(x);
@@ -362,6 +379,7 @@ int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const 
 int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
                    const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
                    int C_audio, h3_bf16* hn, float* v_video, float* v_audio, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   const int na = ranges->count[H3_AUDIO], nv = ranges->count[H3_VIDEO];
@@ -407,6 +425,7 @@ int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x,
 }
 
 int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream) {
+  H3_TRACE();
   if (n < 0) return fail(H3_ERR_SHAPE, "h3_euler_step: n < 0");
   if (n == 0) return ok();
   H3_REQUIRE_PTR(lat);
@@ -418,6 +437,7 @@ int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float si
 
 int h3_text_refine(const h3_dims* dims, const h3_ranges* ranges, float* x, int n_blocks, const float* const* mods,
                    const float* pos, const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (n_blocks < 0) return fail(H3_ERR_SHAPE, "%s: n_blocks must be >= 0", __func__);
@@ -443,6 +463,7 @@ int h3_text_refine(const h3_dims* dims, const h3_ranges* ranges, float* x, int n
 
 int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, h3_bf16* lat_bf16,
                        void* stream) {
+  H3_TRACE();
   if (n < 0) return fail(H3_ERR_SHAPE, "h3_euler_step_bf16: n < 0");
   if (n == 0) return ok();
   H3_REQUIRE_PTR(lat);
@@ -456,6 +477,7 @@ int h3_euler_step_bf16(float* lat, const float* vel, int64_t n, float sigma, flo
 
 int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod, const float* pos,
                      const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (!w) return fail(H3_ERR_NULL, "%s: weights is NULL", __func__);
@@ -488,6 +510,7 @@ int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, con
 }
 
 int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream) {
+  H3_TRACE();
   if (n < 0) return fail(H3_ERR_SHAPE, "h3_exp2_fma_pipe: n < 0");
   if (n == 0) return ok();
   H3_REQUIRE_PTR(x);
@@ -498,6 +521,7 @@ int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream) {
 }
 
 int h3_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  H3_TRACE();
   if (limit_ns == 0 || limit_ns > 10000000000ull)
     return fail(H3_ERR_SHAPE, "h3_selftest_wait_timeout: limit must be in (0, 10 s]");
   cudaError_t e = launch_wait_timeout_selftest((unsigned long long)limit_ns, static_cast<cudaStream_t>(stream));
@@ -506,6 +530,7 @@ int h3_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
 }
 
 int h3_device_status(void* stream, int* code_out) {
+  H3_TRACE();
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: synchronize");
   int code = 0;

@@ -40,6 +40,7 @@ extern "C" {
 
 int h3_quantize_rows_e4m3(const h3_bf16* in, int64_t ld_in, int rows, int cols, h3_e4m3* q, int64_t ld_q,
                           float* scale, void* stream) {
+  H3_TRACE();
   if (rows < 0 || cols <= 0 || cols % 8 || ld_in < cols || ld_q < cols || ld_in % 8 || ld_q % 8)
     return fail(H3_ERR_SHAPE, "%s: need rows >= 0, cols > 0, cols, ld_in, ld_q multiples of 8, ld >= cols",
                 __func__);
@@ -55,6 +56,7 @@ int h3_quantize_rows_e4m3(const h3_bf16* in, int64_t ld_in, int rows, int cols, 
 
 int h3_adaln_norm_modulate_e4m3(const h3_dims* dims, const h3_ranges* ranges, const float* x, const float* mod,
                                 int branch, h3_e4m3* xq, float* xs, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (branch != H3_MSA && branch != H3_MLP) return fail(H3_ERR_SHAPE, "%s: branch must be H3_MSA or H3_MLP", __func__);
@@ -71,6 +73,7 @@ int h3_adaln_norm_modulate_e4m3(const h3_dims* dims, const h3_ranges* ranges, co
 int h3_qkv_qknorm_mrope_e4m3(const h3_dims* dims, const h3_ranges* ranges, const h3_e4m3* xq, const float* xs,
                              const h3_e4m3* Wq, const float* Ws, const h3_bf16* qn_w, const h3_bf16* kn_w,
                              const float* pos, int flags, h3_bf16* q, h3_bf16* k, h3_bf16* v, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
@@ -94,6 +97,7 @@ int h3_qkv_qknorm_mrope_e4m3(const h3_dims* dims, const h3_ranges* ranges, const
 int h3_gated_residual_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_e4m3* oq,
                            const float* os, const h3_e4m3* Wq, const float* Ws, const float* mod, int branch,
                            void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (branch != H3_MSA && branch != H3_MLP) return fail(H3_ERR_SHAPE, "%s: branch must be H3_MSA or H3_MLP", __func__);
@@ -117,6 +121,7 @@ size_t h3_ffn_e4m3_workspace_bytes(const h3_dims* dims, int L_pad) {
 int h3_ffn_swiglu_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_e4m3* xq,
                        const float* xs, const h3_e4m3* Wgu_q, const float* Wgu_s, const h3_e4m3* Wd_q,
                        const float* Wd_s, const float* mod, void* ws, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   H3_REQUIRE_PTR(x);
@@ -150,6 +155,7 @@ int h3_ffn_swiglu_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, c
 int h3_block_forward_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod,
                           const float* pos, const h3_block_weights_e4m3* w, const h3_block_buffers_e4m3* buf,
                           int flags, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (!w) return fail(H3_ERR_NULL, "%s: weights is NULL", __func__);

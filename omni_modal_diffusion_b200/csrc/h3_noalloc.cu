@@ -52,6 +52,7 @@ int static_ws_address(void** out) {
 
 extern "C" int h3_ffn_swiglu_noalloc(const h3_dims* dims, const h3_ranges* ranges, float* x, const h3_bf16* xm,
                                      const h3_bf16* Wgu, const h3_bf16* Wd, const float* mod, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   H3_REQUIRE_PTR(x);

@@ -86,6 +86,7 @@ int h3_sp_make_layout(const h3_dims* dims, const h3_ranges* global, int n_ranks,
 int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3_sp_layout* layout,
                            const h3_bf16* xm, const h3_bf16* Wqkv, const h3_bf16* qn_w, const h3_bf16* kn_w,
                            const float* pos, int flags, const h3_sp_peers* peers, void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(shard, __func__));
   H3_CHECK(check_layout(dims, layout, __func__));
@@ -117,6 +118,7 @@ int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3
 
 int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers, int flags,
                     void* stream) {
+  H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_layout(dims, layout, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))

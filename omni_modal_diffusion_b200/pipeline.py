@@ -193,13 +193,36 @@ class H3Sampler:
         h3.h3_euler_step_bf16(lat_video, st.v_video, sv[s], sv[s + 1], video_bf16, stream=stream)
         h3.h3_euler_step_bf16(lat_audio, st.v_audio, sa[s], sa[s + 1], audio_bf16, stream=stream)
 
-    def run(self, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, n_steps: int, stream=None):
-        """lat_*: fp32 latents at sigma = 1, updated in place; *_bf16: their
-        bf16 copies (the first step's transformer input), kept in step."""
+    def run(self, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, n_steps: int, stream=None,
+            start_step: int = 0, end_step: int | None = None):
+        """lat_*: fp32 latents (at sigma = 1 when start_step is 0), updated in
+        place; *_bf16: their bf16 copies (the next step's transformer input),
+        kept in step.  Runs steps [start_step, end_step) of the n_steps
+        schedule (all of them by default), so that a run can stop after a
+        checkpoint and resume from it."""
         sv = h3.h3_sigma_schedule(n_steps, self.shifts[0])
         sa = h3.h3_sigma_schedule(n_steps, self.shifts[1])
-        for s in range(n_steps):
+        for s in range(start_step, n_steps if end_step is None else end_step):
             self.step(s, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, sv, sa, stream)
+
+    # ---------------------------------------------------------- checkpoint / resume
+    @staticmethod
+    def save_state(path: str, next_step: int, lat_video, lat_audio):
+        """The sampler's whole state: the fp32 latents and the index of the
+        next denoise step (an .npz file).  Weights and modulation are inputs,
+        not state."""
+        np.savez(path, next_step=np.int64(next_step), lat_video=lat_video.detach().cpu().numpy(),
+                 lat_audio=lat_audio.detach().cpu().numpy())
+
+    @staticmethod
+    def load_state(path: str, device):
+        """(next_step, lat_video, lat_audio, video_bf16, audio_bf16) on
+        `device`; the bf16 copies are the latents rounded to nearest, which is
+        what the Euler step writes for the next step."""
+        z = np.load(path)
+        lv = torch.from_numpy(z["lat_video"]).to(device)
+        la = torch.from_numpy(z["lat_audio"]).to(device)
+        return int(z["next_step"]), lv, la, lv.to(torch.bfloat16), la.to(torch.bfloat16)
 
     def launches_per_step(self) -> int:
         st = self.st
