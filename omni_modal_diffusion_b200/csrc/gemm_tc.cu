@@ -27,7 +27,15 @@ constexpr int B_STAGE_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
+// The fp32 store epilogue transposes each 32 x 32 chunk of a warp's rows
+// through shared memory (pitch 36 words: 16-byte rows, conflict-free for the
+// 8-lane phases of 16-byte accesses both ways) so that every global store
+// instruction writes four rows' 128 contiguous bytes each.
+constexpr int EPI_PITCH = 36;
+constexpr int EPI_STAGE_BYTES = 4 * 32 * EPI_PITCH * 4;
+// [1 KB alignment slack][stages][512 B barriers, TMEM slot, RoPE tables][epilogue staging]
+constexpr int MISC_BYTES = 512;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + MISC_BYTES + EPI_STAGE_BYTES;
 
 __device__ __forceinline__ int modality_of(int row, const GemmEpilogue& e) {
 #pragma unroll
@@ -79,7 +87,11 @@ __device__ __forceinline__ void scale_chunk(const GemmEpilogue& e, float* v, int
 }
 
 // ------------------------------------------------------------ epilogues
-__device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb, int m, int n0) {
+// stage: this warp's [32][EPI_PITCH] fp32 buffer; lane = row m - m0 of the
+// warp's 32 consecutive rows.
+__device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb, int m, int n0, float* stage) {
+  const int lane = threadIdx.x & 31;
+  const int m0 = m - lane;
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     const int nc = n0 + c * 32;
@@ -88,14 +100,25 @@ __device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb
     ld_chunk(tb + c * 32, v);
     tmem_wait_ld();
     scale_chunk(e, v, m, nc);
-    if (m < e.M) {
-      float* dst = static_cast<float*>(e.out) + (long)(e.row_off + m) * e.ldo + nc;
-      if (nc + 32 <= e.N) {
+    __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4*>(stage + lane * EPI_PITCH + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    __syncwarp();
+    // lane l: row 4 i + l / 8, columns 4 (l % 8) .. + 3 of the chunk
+    const int sub = lane >> 3, col = nc + 4 * (lane & 7);
+    float* out = static_cast<float*>(e.out);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 4 * i + sub;
+      if (m0 + r >= e.M) continue;
+      const float4 w = *reinterpret_cast<const float4*>(stage + r * EPI_PITCH + 4 * (lane & 7));
+      float* dst = out + (long)(e.row_off + m0 + r) * e.ldo + col;
+      if (col + 4 <= e.N) {
+        *reinterpret_cast<float4*>(dst) = w;
       } else {
-        for (int j = 0; j < 32 && nc + j < e.N; ++j) dst[j] = v[j];
+        const float wv[4] = {w.x, w.y, w.z, w.w};
+        for (int k = 0; k < 4 && col + k < e.N; ++k) dst[k] = wv[k];
       }
     }
   }
@@ -285,6 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + MISC_BYTES);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const GemmEpilogue& e = p.epi;
@@ -402,7 +426,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int m = mt * BM + row_in_tile;
       switch (e.mode) {
-        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN); break;
+        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN, epi_stage + q * 32 * EPI_PITCH); break;
         case EPI_GATED_RESID: epi_gated_resid(e, tb, m, nt * BN); break;
         case EPI_SWIGLU: epi_swiglu(e, tb, m, nt); break;
         case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair); break;
@@ -435,7 +459,7 @@ constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = 128 * BK * 2;             // 16 KB
 constexpr int P_B_BYTES = 128 * BK * 2;             // 16 KB (half of the 256 columns)
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 512;
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + MISC_BYTES + EPI_STAGE_BYTES;
 
 template <bool F8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
@@ -455,6 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + MISC_BYTES);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
@@ -581,7 +606,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int m = mt * 256 + (int)rank * 128 + row_in_tile;
       switch (e.mode) {
-        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN); break;
+        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN, epi_stage + q * 32 * EPI_PITCH); break;
         case EPI_GATED_RESID: epi_gated_resid(e, tb, m, nt * BN); break;
         case EPI_SWIGLU: epi_swiglu(e, tb, m, nt); break;
         case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair); break;
