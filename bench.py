@@ -498,6 +498,8 @@ def run_sampler(args, w):
               for _ in range(args.layers)]
     weights_gb = sum(t.numel() * 2 for b_ in blocks for t in b_.values()) / 1e9
     smp = H3Sampler(w, io, blocks, device=dev, e4m3=args.e4m3)
+    if args.e4m3:
+        del blocks  # the sampler keeps the e4m3 copies only
     L = smp.st.ranges.L
     n_total = args.warmup + args.steps
     text = rnd(w.n_text, w.D_text)

@@ -156,7 +156,8 @@ class H3Sampler:
 
     e4m3=True runs the blocks with their four GEMMs on e4m3 operands
     (h3_block_forward_e4m3): each block's weights are quantised once on the
-    GPU here and the bf16 block weights are released."""
+    GPU here and only the e4m3 copies are kept (the caller may drop its bf16
+    block weights afterwards)."""
 
     def __init__(self, w: Workload, io_weights: dict, block_weights: list, device="cuda",
                  shift_video: float = 12.0, shift_audio: float = 3.0, e4m3: bool = False):
@@ -165,10 +166,7 @@ class H3Sampler:
         self.e4m3 = e4m3
         if e4m3:
             st.alloc_e4m3()
-            self.block_tensors = []
-            for i in range(len(block_weights)):
-                self.block_tensors.append(st.quantize_block_weights_e4m3(block_weights[i]))
-                block_weights[i] = None                # drop the bf16 copy as soon as it is quantised
+            self.block_tensors = [st.quantize_block_weights_e4m3(Wb) for Wb in block_weights]
             torch.cuda.synchronize(st.device)
             self.blocks = [h3.block_weights_e4m3(Wb) for Wb in self.block_tensors]
             self.bufs = h3.block_buffers_e4m3({"xq": st.xq, "xs": st.xs, "q": st.q, "k": st.k, "v": st.v,
