@@ -15,8 +15,9 @@
 //              per thread: S from TMEM, online softmax in the log2 domain
 //              with a lazily moved reference max (O is rescaled in TMEM only
 //              when the row max grows by more than 2^8), P written back over
-//              S in TMEM as packed bf16 and consumed from there by the PV
-//              MMA, finally O / l to global memory.
+//              S in TMEM as packed bf16 in two halves of 64 keys, each
+//              released to the PV MMA as soon as it is stored, finally O / l
+//              to global memory.
 // TMEM (512 columns): tile t owns columns [256t, 256t + 128) for S / P and
 // [256t + 128, 256t + 256) for O.
 #include "h3_internal.cuh"
@@ -76,9 +77,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* v_empty = bars + 7;   // [2] per V stage: freed after the tile's last PV MMA
   uint64_t* s_full = bars + 9;    // [2] per query tile
   uint64_t* o_final = bars + 11;  // [2] per query tile
-  uint64_t* p_full = bars + 13;   // [2] per query tile: P in TMEM (4 warp arrivals)
-  uint64_t* drain = bars + 15;    // the MMA issuer's last commit before teardown
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* p_full = bars + 13;   // [2 tiles][2 halves of the key tile]: P half in TMEM (4 warp arrivals)
+  uint64_t* drain = bars + 17;    // the MMA issuer's last commit before teardown
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -96,7 +97,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);
+      mbar_init(&p_full[2 * s], 4);
+      mbar_init(&p_full[2 * s + 1], 4);
       mbar_init(&o_final[s], 1);
     }
     mbar_init(drain, 1);
@@ -163,13 +165,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       umma_commit(&s_full[t]);
     };
-    // O_t += P_t V_j, P_t (bf16, two per column) read from TMEM where S_t was
-    auto issue_pv = [&](int t, int j) {
+    // O_t += P_t V_j for keys [64 hf, 64 hf + 64): P_t (bf16, two per column)
+    // read from TMEM columns [32 hf, 32 hf + 32) where S_t was
+    auto issue_pv_half = [&](int t, int j, int hf) {
       const uint64_t vd = v_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = hf * 4 + k4;
         umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_o,
                          (j | kk) != 0 ? 1u : 0u);
+      }
     };
     bool ok = MMA_WAIT_WARP(q_full, 0) && MMA_WAIT_WARP(&k_full[0], 0);
     if (ok) {
@@ -181,10 +186,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int j = 0; j < nkv && ok; ++j) {
       const bool more = j + 1 < nkv;
       for (int t = 0; t < 2 && ok; ++t) {
-        if (!MMA_WAIT_WARP(&p_full[t], j & 1)) { ok = false; break; }
-        if (t == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(t, j);
+        // P is released in two halves: PV on keys [0, 64) runs while the
+        // softmax warps still take the second half's exponentials
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!MMA_WAIT_WARP(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
+          if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv_half(t, j, hf);
+        }
+        if (!ok) break;
         if (more) {
           if (t == 0) {
             if (!MMA_WAIT_WARP(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
@@ -273,12 +283,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tS + hf * 32, pk);
-        if (hf == 1) {
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[t]);
-        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[2 * t + hf]);
       }
       float a0, a1, a2, a3;
       f2_unpack(acc[0], a0, a1);
