@@ -69,11 +69,11 @@ def bytes_per_call(w, L, Lp):
 # kernel changes (see profiles/).
 TRAFFIC = {
     # mean over the block's QKV, out-projection, FFN gate/up and FFN down
-    # launches (6.202 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel"): 1.550e9,
-    # the same four launches with e4m3 operands (2.640 GB / 4),
+    # launches (6.156 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    ("768sq_2s", "gemm_tc_kernel"): 1.539e9,
+    # the same four launches with e4m3 operands (2.679 GB / 4),
     # profiles/gemm_tc_kernel_e4m3_768sq_2s.md
-    ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.660e9,
+    ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.670e9,
     # profiles/attention_tc_kernel_768sq_2s.md
     ("768sq_2s", "attention_tc_kernel"): 0.4348e9,
 }

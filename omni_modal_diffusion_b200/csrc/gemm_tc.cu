@@ -124,13 +124,15 @@ __device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb
   }
 }
 
-__device__ __forceinline__ void epi_gated_resid(const GemmEpilogue& e, uint32_t tb, int m, int n0) {
+// Chunks [c_lo, c_hi) of 32 accumulator columns (all BN / 32 by default).
+__device__ __forceinline__ void epi_gated_resid(const GemmEpilogue& e, uint32_t tb, int m, int n0, int c_lo = 0,
+                                                int c_hi = BN / 32) {
   const int row = e.row_off + m;
   const int mod_id = (m < e.M) ? modality_of(row, e) : -1;
   const float* gate = e.mod + (long)((mod_id < 0 ? 0 : mod_id) * 6 + e.gate_slot) * e.D;
   float* xrow = static_cast<float*>(e.out) + (long)row * e.ldo;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
+  for (int c = c_lo; c < c_hi; ++c) {
     const int nc = n0 + c * 32;
     if (nc >= e.N) break;
     float v[32];
@@ -156,12 +158,13 @@ __device__ __forceinline__ void epi_gated_resid(const GemmEpilogue& e, uint32_t 
   }
 }
 
-__device__ __forceinline__ void epi_swiglu(const GemmEpilogue& e, uint32_t tb, int m, int nt) {
+__device__ __forceinline__ void epi_swiglu(const GemmEpilogue& e, uint32_t tb, int m, int nt, int c_lo = 0,
+                                           int c_hi = 4) {
   // columns [0,128) of the accumulator hold gate, [128,256) hold up, for
-  // output columns nt*128 + [0,128)
+  // output columns nt*128 + [0,128); chunks [c_lo, c_hi) of 32 of them
   bf16* dst = static_cast<bf16*>(e.out) + (long)m * e.ldo + (long)nt * 128;
 #pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
+  for (int c = c_lo; c < c_hi; ++c) {
     float g[32], u[32];
     ld_chunk(tb + c * 32, g);
     ld_chunk(tb + 128 + c * 32, u);
@@ -199,8 +202,11 @@ __device__ __forceinline__ void rope_sincos(float a, float* s, float* c) {
   __sincosf(r, s, c);
 }
 
+// Heads [h_lo, h_hi) of the tile's two 128-column heads.  Two passes over
+// TMEM per head: the sum of squares of the 128 values, then chunk by chunk
+// normalise, rotate and store (no 128-value array in registers).
 __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int m, int n0, const float* freq,
-                                        const uint8_t* axis_of_pair) {
+                                        const uint8_t* axis_of_pair, int h_lo = 0, int h_hi = 2) {
   float p3[3] = {0.f, 0.f, 0.f};
   if (m < e.L_pad) {
     p3[0] = e.pos[(long)m * 3 + 0];
@@ -208,43 +214,29 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
     p3[2] = e.pos[(long)m * 3 + 2];
   }
 #pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
+  for (int half = h_lo; half < h_hi; ++half) {
     const int n = n0 + half * 128;
     if (n >= e.N) break;  // uniform
     const int part = n / e.I;
     const int h = (n % e.I) / 128;
-    float v[128];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) ld_chunk(tb + half * 128 + c * 32, v + c * 32);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 4; ++c) scale_chunk(e, v + c * 32, m, n + c * 32);
+    const uint32_t th = tb + half * 128;
+    float inv = 1.0f;
+    const bf16* w = part == 0 ? e.qn_w : e.kn_w;
     if (part < 2) {
       float ss = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        ld_chunk(th + c * 32, v);
+        tmem_wait_ld();
+        scale_chunk(e, v, m, n + c * 32);
 #pragma unroll
-      for (int d = 0; d < 128; ++d) ss = fmaf(v[d], v[d], ss);
-      const float inv = rsqrtf(ss * (1.0f / 128.0f) + e.eps_qk);
-      const bf16* w = part == 0 ? e.qn_w : e.kn_w;
-#pragma unroll
-      for (int d = 0; d < 128; d += 8) {
-        const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w + d));
-        const bf16* wb = reinterpret_cast<const bf16*>(&wv);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[d + j] = v[d + j] * inv * __bfloat162float(wb[j]);
+        for (int d = 0; d < 32; ++d) ss = fmaf(v[d], v[d], ss);
       }
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int ax = axis_of_pair[i];
-        const float pa = ax == 0 ? p3[0] : (ax == 1 ? p3[1] : p3[2]);
-        float s, c;
-        rope_sincos(pa * freq[i], &s, &c);
-        const float a = v[2 * i], b = v[2 * i + 1];
-        v[2 * i] = a * c - b * s;
-        v[2 * i + 1] = a * s + b * c;
-      }
+      inv = rsqrtf(ss * (1.0f / 128.0f) + e.eps_qk);
     }
+    bf16* dst = nullptr;
     if (m < e.M) {
-      bf16* dst;
       if (e.sp_n > 0) {  // sequence parallel: straight into the head group's rank
         const int g = h / e.sp_heads, hl = h - g * e.sp_heads;
         bf16* base = part == 0 ? e.sp_q[g] : (part == 1 ? e.sp_k[g] : e.sp_v[g]);
@@ -253,14 +245,43 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
         bf16* base = part == 0 ? e.q : (part == 1 ? e.k : e.v);
         dst = base + ((long)h * e.L_pad + m) * 128;
       }
+    }
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      ld_chunk(th + c * 32, v);
+      tmem_wait_ld();
+      scale_chunk(e, v, m, n + c * 32);
+      if (part < 2) {
 #pragma unroll
-      for (int d = 0; d < 128; d += 8) {
-        uint4 o;
-        o.x = pack_bf16x2(v[d], v[d + 1]);
-        o.y = pack_bf16x2(v[d + 2], v[d + 3]);
-        o.z = pack_bf16x2(v[d + 4], v[d + 5]);
-        o.w = pack_bf16x2(v[d + 6], v[d + 7]);
-        *reinterpret_cast<uint4*>(dst + d) = o;
+        for (int d = 0; d < 32; d += 8) {
+          const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w + c * 32 + d));
+          const bf16* wb = reinterpret_cast<const bf16*>(&wv);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[d + j] = v[d + j] * inv * __bfloat162float(wb[j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int ip = c * 16 + i;  // pair index within the head
+          const int ax = axis_of_pair[ip];
+          const float pa = ax == 0 ? p3[0] : (ax == 1 ? p3[1] : p3[2]);
+          float sn, cs;
+          rope_sincos(pa * freq[ip], &sn, &cs);
+          const float a = v[2 * i], bb = v[2 * i + 1];
+          v[2 * i] = a * cs - bb * sn;
+          v[2 * i + 1] = a * sn + bb * cs;
+        }
+      }
+      if (dst) {
+#pragma unroll
+        for (int d = 0; d < 32; d += 8) {
+          uint4 o;
+          o.x = pack_bf16x2(v[d], v[d + 1]);
+          o.y = pack_bf16x2(v[d + 2], v[d + 3]);
+          o.z = pack_bf16x2(v[d + 4], v[d + 5]);
+          o.w = pack_bf16x2(v[d + 6], v[d + 7]);
+          *reinterpret_cast<uint4*>(dst + c * 32 + d) = o;
+        }
       }
     }
   }
@@ -455,14 +476,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // shared memory, and the leader CTA (rank 0) issues M = 256 MMAs that read
 // both CTAs' operands and leave each CTA's 128 result rows in its own TMEM.
 // Per CTA this stages 32 KB per 64-deep K step instead of 48 KB.
-constexpr int P_STAGES = 6;
+#ifndef H3_GEMM_PAIR_STAGES
+#define H3_GEMM_PAIR_STAGES 6
+#endif
+constexpr int P_STAGES = H3_GEMM_PAIR_STAGES;
 constexpr int P_A_BYTES = 128 * BK * 2;             // 16 KB
 constexpr int P_B_BYTES = 128 * BK * 2;             // 16 KB (half of the 256 columns)
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + MISC_BYTES + EPI_STAGE_BYTES;
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + MISC_BYTES;
+// Warp 0 TMA, warp 1 MMA (leader CTA), warps 2-9 epilogue: two warps per TMEM
+// lane quarter, each taking half of the tile's 256 columns, so that one
+// warp's loads and stores overlap the other's arithmetic.  With e4m3 operands
+// (half the MMA time per tile) one epilogue warp per quarter bounded the QKV
+// GEMM (epilogue busy 20.3K of the MMAs' 21.5K SM clocks per tile) and the
+// out-projection (34K against 29K).
+constexpr int P_NUM_THREADS = 320;
 
 template <bool F8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ GemmProblem p) {
   constexpr int KSTEP = F8 ? 2 * BK : BK;  // elements per stage
@@ -479,7 +510,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
-  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + MISC_BYTES);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
@@ -494,7 +524,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);   // the leader's commit, delivered to both CTAs
-      mbar_init(&tempty[a], 8);  // 4 epilogue warps in each CTA (leader's copy used)
+      mbar_init(&tempty[a], 16);  // 8 epilogue warps in each CTA (leader's copy used)
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -591,7 +621,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(drain, 0);
     }
   } else {
-    const int q = warp & 3;
+    const int q = warp & 3;     // TMEM lane quarter
+    const int sub = (warp - 2) >> 2;  // which half of the tile's columns
     const int row_in_tile = q * 32 + lane;
     const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
     int acc = 0;
@@ -605,12 +636,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int m = mt * 256 + (int)rank * 128 + row_in_tile;
-      switch (e.mode) {
-        case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN, epi_stage + q * 32 * EPI_PITCH); break;
-        case EPI_GATED_RESID: epi_gated_resid(e, tb, m, nt * BN); break;
-        case EPI_SWIGLU: epi_swiglu(e, tb, m, nt); break;
-        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair); break;
-        case EPI_UNPATCH: epi_unpatch(e, tb, m, nt * BN); break;
+      switch (e.mode) {  // the modes the launcher routes here
+        case EPI_GATED_RESID:
+          // the fp32 residual read-modify-write: split between the two
+          // warps only where the MMAs of a tile are short, e4m3 operands and
+          // K <= 8192 (out-projection 0.244 -> 0.236 ms at 7,904 tokens;
+          // split, the e4m3 FFN down-projection took 3.6% more cycles and the
+          // bf16 out-projection 0.416 -> 0.427 ms); else one warp per quarter
+          // takes all 256 columns
+          if (F8 && p.K <= 8192)
+            epi_gated_resid(e, tb, m, nt * BN, sub * 4, sub * 4 + 4);
+          else if (sub == 0)
+            epi_gated_resid(e, tb, m, nt * BN);
+          break;
+        case EPI_SWIGLU: epi_swiglu(e, tb, m, nt, sub * 2, sub * 2 + 2); break;
+        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair, sub, sub + 1); break;
         default: break;
       }
       tc_fence_before();
@@ -738,7 +778,8 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
   // 5.33 -> 1.27 / 5.24 ms; FFN gate/up and down 7% / 13% and 6% / 12% fewer
   // SM cycles (ncu, clock-independent).  The input projections and the heads
   // (small M or N) stay on the one-CTA kernel.
-  if (H3_GEMM_PAIR && p.pair == 1 && p.M > 128) {
+  const bool pair_mode = p.epi.mode == EPI_QKV || p.epi.mode == EPI_GATED_RESID || p.epi.mode == EPI_SWIGLU;
+  if (H3_GEMM_PAIR && p.pair == 1 && p.M > 128 && pair_mode) {
     static unsigned long long attr2_done[2] = {0, 0};
     const void* k2 = f8 ? reinterpret_cast<const void*>(gemm_detail::gemm_tc2_kernel<true>)
                         : reinterpret_cast<const void*>(gemm_detail::gemm_tc2_kernel<false>);
@@ -755,10 +796,10 @@ cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream) {
     const int max_pairs = num_sms() / 2;
     const int pairs = pair_tiles < max_pairs ? pair_tiles : max_pairs;
     if (f8)
-      gemm_detail::gemm_tc2_kernel<true><<<2 * pairs, gemm_detail::NUM_THREADS, gemm_detail::P_SMEM_BYTES, stream>>>(
+      gemm_detail::gemm_tc2_kernel<true><<<2 * pairs, gemm_detail::P_NUM_THREADS, gemm_detail::P_SMEM_BYTES, stream>>>(
           tmA, tmB, q2);
     else
-      gemm_detail::gemm_tc2_kernel<false><<<2 * pairs, gemm_detail::NUM_THREADS, gemm_detail::P_SMEM_BYTES,
+      gemm_detail::gemm_tc2_kernel<false><<<2 * pairs, gemm_detail::P_NUM_THREADS, gemm_detail::P_SMEM_BYTES,
                                             stream>>>(tmA, tmB, q2);
     return cudaGetLastError();
   }
