@@ -65,16 +65,15 @@ def bytes_per_call(w, L, Lp):
 
 
 # DRAM bytes (read + write) per launch from one ncu capture of the kernel on
-# this workload, valid for the kernel as it was when captured; None once the
-# kernel changes (see profiles/).
+# this workload (dram__bytes_read.sum + dram__bytes_write.sum), valid for the
+# kernel as it was when captured.
 TRAFFIC = {
     # mean over the block's QKV, out-projection, FFN gate/up and FFN down
-    # launches (6.156 GB / 4), profiles/gemm_tc_kernel_768sq_2s.md
+    # launches (6.156 GB / 4)
     ("768sq_2s", "gemm_tc_kernel"): 1.539e9,
-    # the same four launches with e4m3 operands (2.679 GB / 4),
-    # profiles/gemm_tc_kernel_e4m3_768sq_2s.md
+    # the same four launches with e4m3 operands (2.679 GB / 4)
     ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.670e9,
-    # profiles/attention_tc_kernel_768sq_2s.md
+    # one attention launch
     ("768sq_2s", "attention_tc_kernel"): 0.4348e9,
 }
 

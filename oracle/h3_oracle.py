@@ -18,7 +18,7 @@ Sources (page title, section):
            worked example
   [0539]   "H3's omni-modal ambition" (0539edu.com), scheduler sigma shifts
 
-Readings where the pages are silent or garbled (each listed in the design doc):
+Readings adopted where the pages are silent or garbled:
   G1 packing order text -> audio -> video; G2 latent frames 1 + (T-1)//4;
   G3 RoPE split t/h/w = 32/48/48; G4 theta 10000, interleaved pairs;
   G5 positions (video (t,i,j); audio (0.15 k, 0, 0); text (0,0,0));
