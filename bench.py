@@ -329,6 +329,9 @@ def run_ours(args, w):
     block_ms = sum(per_call[c] for c in ("h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
                                          "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu"))
     ln_gbs = by["h3_adaln_norm_modulate"] / (per_call["h3_adaln_norm_modulate"] / 1e3) / 1e9
+    # two launches (video and audio latents); the latents were just written
+    # by the head, so at this size they are read from L2
+    euler_gbs = by["h3_euler_step"] / (per_call["h3_euler_step"] / 1e3) / 1e9
     launches = st.launches_per_step()
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -353,6 +356,7 @@ def run_ours(args, w):
         "per_call_ms": {c: round(v, 4) for c, v in per_call.items()},
         "per_call_tflops": {c: round(v, 1) for c, v in tensor_calls.items()},
         "ln_modulate_gbs": round(ln_gbs, 1), "ln_modulate_frac_hbm": round(ln_gbs / peaks["hbm_gbs"], 4),
+        "euler_gbs": round(euler_gbs, 1), "euler_frac_hbm": round(euler_gbs / peaks["hbm_gbs"], 4),
         "gpu_launches": launches * args.steps,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,
@@ -573,6 +577,11 @@ def run_only(args, w):
         Wgu, Wd = rnd(2 * w.F, w.D, std=0.02), rnd(w.D, w.F, std=0.02)
         ws = torch.empty(Lp, w.F, dtype=torch.bfloat16, device=dev)
         fn = lambda: h3.h3_ffn_swiglu(d, r, x, xm, Wgu, Wd, mod, ws)
+    elif args.only == "euler":
+        # the video and audio latents of the workload, updated in place
+        n_lat = w.T_lat * w.H_lat * w.W_lat * w.C_lat + w.audio_channels * w.n_audio * w.C_audio
+        lat, vel = rnd(n_lat, dt=torch.float32), rnd(n_lat, dt=torch.float32)
+        fn = lambda: h3.h3_euler_step(lat, vel, 0.5, 0.4)
     else:
         x = rnd(Lp, w.D, dt=torch.float32)
         xm = torch.empty(Lp, w.D, dtype=torch.bfloat16, device=dev)
@@ -665,7 +674,7 @@ def main():
     ap.add_argument("--layers", type=int, default=50)
     ap.add_argument("--e4m3", action="store_true",
                     help="the block step with its four GEMMs in e4m3 (a separate line; one GPU)")
-    ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln"],
+    ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln", "euler"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=None, help=f"default {DEFAULT_WORKLOAD}; sampler: 768x1344_5s")
