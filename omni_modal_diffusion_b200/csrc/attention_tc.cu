@@ -13,11 +13,12 @@
 //              tensor core runs the other tile's PV and next S.
 //   Warps 2-5  softmax of query tile 0, warps 6-9 of tile 1, one query row
 //              per thread: S from TMEM, online softmax in the log2 domain
-//              with a lazily moved reference max (O is rescaled in TMEM only
-//              when the row max grows by more than 2^8), P written back over
-//              S in TMEM as packed bf16 in two halves of 64 keys, each
-//              released to the PV MMA as soon as it is stored, finally O / l
-//              to global memory.
+//              against a lazily moved reference (the first key tile's row
+//              max; it moves only when a 64-key half's exponentials sum past
+//              2^16, with O rescaled in TMEM and that half redone), P written
+//              back over S in TMEM as packed bf16 in two halves of 64 keys,
+//              each released to the PV MMA as soon as it is stored, finally
+//              O / l to global memory.
 // TMEM (512 columns): tile t owns columns [256t, 256t + 128) for S / P and
 // [256t + 128, 256t + 256) for O.
 #include "h3_internal.cuh"
@@ -26,6 +27,18 @@
 namespace h3 {
 
 namespace attn_detail {
+// 8-column TMEM load / store (32 lanes x 8 columns), for the rare rescale of
+// O where the softmax registers are all live
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 constexpr int NUM_THREADS = 320;
 constexpr int TILE = 128;
 constexpr int HALF_BYTES = TILE * 64 * 2;   // 128 rows x 64 bf16 = 16 KB
@@ -36,7 +49,11 @@ constexpr int SMEM_V = SMEM_K + 2 * TILE_BYTES;  // 2 stages
 constexpr int SMEM_BAR = SMEM_V + 2 * TILE_BYTES;
 constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
 constexpr int TMEM_COLS = 512;
-constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// A 64-key half whose exponentials (against the current reference) sum past
+// this moves the reference: every p of an accepted half is <= 2^16, so p, the
+// row sum and O stay far from the fp32 range (and bf16 P keeps its relative
+// precision at any scale).
+constexpr float P_HALF_SUM_LIMIT = 65536.0f;
 // How the MMA issuer waits: polling (1) or suspending try_wait (0).  The
 // suspending wait leaves the issue slots of its sub-partition to the softmax
 // warps that share it: 1.486 vs 1.499 ms at 7,904 tokens, equal at 32,160.
@@ -79,7 +96,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* o_final = bars + 11;  // [2] per query tile
   uint64_t* p_full = bars + 13;   // [2 tiles][2 halves of the key tile]: P half in TMEM (4 warp arrivals)
   uint64_t* drain = bars + 17;    // the MMA issuer's last commit before teardown
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* pv0_done = bars + 18; // [2] per query tile: PV on the first key half complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -99,6 +117,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[2 * s], 4);
       mbar_init(&p_full[2 * s + 1], 4);
+      mbar_init(&pv0_done[s], 1);
       mbar_init(&o_final[s], 1);
     }
     mbar_init(drain, 1);
@@ -193,6 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv_half(t, j, hf);
+          if (hf == 0) umma_commit(&pv0_done[t]);
         }
         if (!ok) break;
         if (more) {
@@ -228,51 +248,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_wait_ld();
 
       const int valid = L - j * TILE;  // keys [0, valid) of this tile are real
-      const bool full = valid >= TILE;
-      float mx = -INFINITY;
-      if (full) {
+      if (valid < TILE) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      // row max over keys [c0, c0 + n)
+      auto row_max = [&](int c0, int n) {
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
+        for (int c = c0; c < c0 + n; c += 8) {
           m4[0] = max3f(m4[0], s[c], s[c + 1]);
           m4[1] = max3f(m4[1], s[c + 2], s[c + 3]);
           m4[2] = max3f(m4[2], s[c + 4], s[c + 5]);
           m4[3] = max3f(m4[3], s[c + 6], s[c + 7]);
         }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          if (c >= valid) s[c] = -INFINITY;
-          mx = fmaxf(mx, s[c]);
-        }
-      }
-      const float m_new = fmaxf(m_ref, mx * scale_log2);
-      const bool move = (m_new - m_ref) > RESCALE_THRESHOLD;  // true at j == 0 (m_ref = -inf)
-      const float alpha = move ? ex2_approx(m_ref - m_new) : 1.0f;
-      if (move) m_ref = m_new;
-      // O_t is stable here: PV_t,j-1 completed before S_t,j was signalled
-      if (j > 0 && __any_sync(0xffffffffu, move)) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float o[32];
-          tmem_ld32(tO + c * 32, reinterpret_cast<uint32_t*>(o));
-          tmem_wait_ld();
-#pragma unroll
-          for (int d = 0; d < 32; ++d) o[d] *= alpha;
-          tmem_st32(tO + c * 32, reinterpret_cast<const uint32_t*>(o));
-        }
-      }
-      // p = 2^(s * scale_log2 - m_ref) on the MUFU unit (masked keys, -inf,
-      // give exactly 0)
+        return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      };
+      // The reference m_ref is the row max of the first key tile, and moves
+      // only when a later tile would overflow against it: the exponentials
+      // of each 64-key half are taken against the current reference, and a
+      // half whose row sum exceeds 2^16 (some p > 2^16) is redone against
+      // that half's row max, with O and the sums rescaled first.  A half that
+      // passed the check lies within 2^16 of the reference, so it stays in
+      // range when the reference moves up.  No per-tile row max otherwise.
+      if (j == 0) m_ref = row_max(0, 128) * scale_log2;
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
-      const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
-      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-      // P for keys [64 hf, 64 hf + 64) goes to TMEM columns [32 hf, 32 hf + 32)
-      // (it only overwrites S columns already in registers)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
+      // p = 2^(s * scale_log2 - m_ref) on the MUFU unit (masked keys, -inf,
+      // give exactly 0); returns this row's sum over the half
+      auto exp_half = [&](int hf, uint32_t* pk) {
+        const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+        uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const int cc = hf * 64 + c;
@@ -282,16 +288,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_pack(p0, p1));
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
+        float a0, a1, a2, a3;
+        f2_unpack(acc[0], a0, a1);
+        f2_unpack(acc[1], a2, a3);
+        return (a0 + a1) + (a2 + a3);
+      };
+      float hsum[2];
+      // P for keys [64 hf, 64 hf + 64) goes to TMEM columns [32 hf, 32 hf + 32)
+      // (it only overwrites S columns already in registers)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+        float hs = exp_half(hf, pk);
+        if (j > 0 && __any_sync(0xffffffffu, !(hs <= P_HALF_SUM_LIMIT))) {
+          // this half's scores again, from TMEM: P has not overwritten them
+          // (P of keys [0, 64) goes to columns [0, 32))
+          tmem_ld32(tS + hf * 64, reinterpret_cast<uint32_t*>(s + hf * 64));
+          tmem_ld32(tS + hf * 64 + 32, reinterpret_cast<uint32_t*>(s + hf * 64 + 32));
+          tmem_wait_ld();
+          if (valid < TILE) {
+#pragma unroll
+            for (int c = hf * 64; c < hf * 64 + 64; ++c)
+              if (c >= valid) s[c] = -INFINITY;
+          }
+          const float m_new = fmaxf(m_ref, row_max(hf * 64, 64) * scale_log2);
+          const float a = ex2_approx(m_ref - m_new);  // 1 where the reference holds
+          m_ref = m_new;
+          // O must hold every PV issued against the old reference before it
+          // is rescaled: PV_t,j-1 completed before S_t,j was signalled; the
+          // first half of PV_t,j has its own barrier
+          if (hf == 1) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&pv0_done[t], j & 1))) { ok = false; break; }
+            tc_fence_after();
+            hsum[0] *= a;
+          }
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[8];
+            tmem_ld8(tO + c * 8, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int d = 0; d < 8; ++d) o[d] = __float_as_uint(__uint_as_float(o[d]) * a);
+            tmem_st8(tO + c * 8, o);
+          }
+          tmem_wait_st();
+          l_sum *= a;
+          hs = exp_half(hf, pk);
+        }
+        hsum[hf] = hs;
         tmem_st32(tS + hf * 32, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[2 * t + hf]);
       }
-      float a0, a1, a2, a3;
-      f2_unpack(acc[0], a0, a1);
-      f2_unpack(acc[1], a2, a3);
-      l_sum = fmaf(l_sum, alpha, (a0 + a1) + (a2 + a3));
+      if (!ok) break;
+      l_sum += hsum[0] + hsum[1];
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
     const int qt = t == 0 ? qt0 : qt1;

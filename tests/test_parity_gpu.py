@@ -307,6 +307,40 @@ def test_attention_edge_lengths():
             assert np.allclose(got[0], qkv[2][:, 0, :].reshape(-1), rtol=1e-2, atol=1e-2)
 
 
+@pytest.mark.parametrize("kind", ["ramp", "spike_last", "spike_second_half"])
+def test_attention_reference_moves(kind):
+    """Scores that grow along the keys, far past the first key tile's row max:
+    the kernel's reference (the first tile's max) must move, with O and the
+    running sums rescaled, in either 64-key half of a tile.  ramp: key norms
+    grow 7x over the sequence; spike_last: the last (partial) key tile scaled
+    30x (p would overflow fp32 against the old reference); spike_second_half:
+    keys [64, 128) of an interior tile scaled 30x (the first half's PV is
+    already issued when the second half moves the reference)."""
+    H, L = 4, 1000
+    d = h3.make_dims(320, H, 896)
+    rg = h3.h3_make_ranges(L, 0, 0)
+    Lp = rg.L_pad
+    rng = np.random.default_rng({"ramp": 1, "spike_last": 2, "spike_second_half": 3}[kind])
+    q, k, v = (rng.standard_normal((H, Lp, 128), dtype=np.float32) for _ in range(3))
+    if kind == "ramp":
+        k *= (1 + 6 * np.arange(Lp, dtype=np.float32) / L)[None, :, None]
+    elif kind == "spike_last":
+        k[:, (L - 1) // 128 * 128:] *= 30
+    else:
+        k[:, 3 * 128 + 64: 4 * 128] *= 30
+    q, k, v = (S.bf16_round(a) for a in (q, k, v))
+    for a in (q, k, v):
+        a[:, L:, :] = 0
+    o = torch.empty(Lp, H * 128, dtype=torch.bfloat16, device=DEV)
+    h3.h3_attention(d, rg, *(to_dev_bf16(a, DEV) for a in (q, k, v)), o)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    got = to_np(o)
+    ref = O.attention(*(a[:, :L, :].transpose(1, 0, 2).astype(np.float64) for a in (q, k, v)))
+    check_close(got[:L], ref, f"attention ({kind})")
+    assert np.all(got[L:] == 0)
+
+
 # ---------------------------------------------------------------- full sizes, sampled outputs
 
 FULL = [S.WORKLOADS["768sq_2s"], S.WORKLOADS["768x1344_5s"]]
