@@ -405,6 +405,10 @@ def run_e4m3(args, w):
              "h3_quantize_rows_e4m3", "h3_gated_residual_e4m3", "h3_adaln_norm_modulate_e4m3#2",
              "h3_ffn_swiglu_e4m3", "h3_head_unpack", "h3_euler_step"]
 
+    # --qk-e4m3: q, k cross to attention as e4m3 codes (H3_QK_E4M3)
+    qk_flags = h3.H3_QK_NORM_ROPE_IN_QKV | (h3.H3_QK_E4M3 if args.qk_e4m3 else 0)
+    qb, kb = (st.q8, st.k8) if args.qk_e4m3 else (st.q, st.k)
+
     def step(i, ev=None):
         s = i % 8
         mark = (lambda k, j: ev[k][j].record(stream)) if ev is not None else (lambda k, j: None)
@@ -413,9 +417,11 @@ def run_e4m3(args, w):
         mark(1, 0); h3.h3_adaln_norm_modulate_e4m3(d, r, st.x, mod, h3.H3_MSA, st.xq, st.xs); mark(1, 1)
         mark(2, 0)
         h3.h3_qkv_qknorm_mrope_e4m3(d, r, st.xq, st.xs, W8["Wqkv"], W8["Wqkv_s"], W8["qn_w"], W8["kn_w"], st.pos,
-                                    st.q, st.k, st.v)
+                                    qb, kb, st.v, flags=qk_flags)
         mark(2, 1)
-        mark(3, 0); h3.h3_attention(d, r, st.q, st.k, st.v, st.o); mark(3, 1)
+        mark(3, 0)
+        h3.h3_attention(d, r, qb, kb, st.v, st.o, qn_w=W8["qn_w"], kn_w=W8["kn_w"], flags=qk_flags)
+        mark(3, 1)
         mark(4, 0); h3.h3_quantize_rows_e4m3(st.o, st.oq, st.os); mark(4, 1)
         mark(5, 0); h3.h3_gated_residual_e4m3(d, r, st.x, st.oq, st.os, W8["Wo"], W8["Wo_s"], mod); mark(5, 1)
         mark(6, 0); h3.h3_adaln_norm_modulate_e4m3(d, r, st.x, mod, h3.H3_MLP, st.xq, st.xs); mark(6, 1)
@@ -457,7 +463,8 @@ def run_e4m3(args, w):
     gemm_tf = sum(gemm.values()) / (gemm_ms / 1e3) / 1e12
     block_ms = sum(per_call[c] for c in calls[1:8])
     return {
-        "metric": "packed tokens/s per Omni block (e4m3 GEMMs, bf16 attention, 1×B200)",
+        "metric": ("packed tokens/s per Omni block (e4m3 GEMMs, e4m3 Q K^T, bf16 P V, 1×B200)" if args.qk_e4m3
+                   else "packed tokens/s per Omni block (e4m3 GEMMs, bf16 attention, 1×B200)"),
         "value": round(L / (ms_step / 1e3), 1), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3 GEMMs (fp32 accumulate), bf16 attention",
@@ -500,7 +507,7 @@ def run_sampler(args, w):
                "Wo": rnd(w.D, w.I, std=0.02), "Wgu": rnd(2 * w.F, w.D, std=0.02), "Wd": rnd(w.D, w.F, std=0.02)}
               for _ in range(args.layers)]
     weights_gb = sum(t.numel() * 2 for b_ in blocks for t in b_.values()) / 1e9
-    smp = H3Sampler(w, io, blocks, device=dev, e4m3=args.e4m3)
+    smp = H3Sampler(w, io, blocks, device=dev, e4m3=args.e4m3, qk_e4m3=args.qk_e4m3)
     if args.e4m3:
         del blocks  # the sampler keeps the e4m3 copies only
     L = smp.st.ranges.L
@@ -529,7 +536,8 @@ def run_sampler(args, w):
     assert h3.h3_device_status() == 0
     ms = a.elapsed_time(b) / args.steps
     fl = block_flops(w, L) * args.layers
-    kind = "e4m3 GEMMs, bf16 attention" if args.e4m3 else "bf16"
+    kind = ("e4m3 GEMMs, e4m3 Q K^T, bf16 P V" if args.qk_e4m3 else "e4m3 GEMMs, bf16 attention") if args.e4m3 \
+        else "bf16"
     return {"metric": f"end-to-end denoise steps/s (layered flow sampler, {kind}, 1xB200)",
             "value": round(1e3 / ms, 4), "unit": "denoise steps/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
@@ -674,6 +682,8 @@ def main():
     ap.add_argument("--layers", type=int, default=50)
     ap.add_argument("--e4m3", action="store_true",
                     help="the block step with its four GEMMs in e4m3 (a separate line; one GPU)")
+    ap.add_argument("--qk-e4m3", action="store_true",
+                    help="with --e4m3: q and k cross to attention as e4m3 codes (Q K^T on e4m3 MMAs)")
     ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln", "euler"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

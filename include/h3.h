@@ -62,6 +62,11 @@ enum h3_branch { H3_MSA = 0, H3_MLP = 1 };
  * in the QKV GEMM epilogue (once per token), and h3_attention consumes the
  * already-rotated q, k.  Required in this version. */
 #define H3_QK_NORM_ROPE_IN_QKV 1
+/* With h3_qkv_qknorm_mrope_e4m3 / h3_attention / h3_block_forward_e4m3 only:
+ * q and k are passed between the QKV call and attention as e4m3 codes (see
+ * the FP8 section), and attention takes S = Q K^T on e4m3 tensor-core MMAs.
+ * P V stays bf16. */
+#define H3_QK_E4M3 2
 
 /* Block dimensions.  head_dim must be 128; I = H * head_dim;
  * rope_t + rope_h + rope_w = head_dim, each even ([gojay] §7.4).
@@ -146,6 +151,9 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
  * non-causal; keys >= L are masked ([shouss] §5).  q, k, v: head-major
  * [H][L_pad][128] bf16 as written by h3_qkv_qknorm_mrope (flags must carry
  * H3_QK_NORM_ROPE_IN_QKV; qn_w, kn_w and pos are then unused and may be NULL).
+ * With flags & H3_QK_E4M3, q and k are the e4m3 codes written by
+ * h3_qkv_qknorm_mrope_e4m3 with that flag (one byte per element) and qn_w,
+ * kn_w are required: the code scales follow from them.
  *   o [L_pad][H*128] bf16, token-major; rows >= L written as 0. */
 int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q, const h3_bf16* k,
                  const h3_bf16* v, const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
@@ -294,8 +302,15 @@ int h3_set_wait_limit_ns(uint64_t ns);
  *     channel (row of the [out][in] weight).  A GEMM then computes
  *     acc[m][n] * a_scale[m] * b_scale[n] and applies the same fused
  *     epilogue as its bf16 counterpart.
- * Attention stays bf16.  Code matrices are row-major bytes; every row length
- * is a multiple of 16 bytes as for the bf16 calls (D % 64, I, F % 128). */
+ * Attention stays bf16 unless H3_QK_E4M3 is set: then q and k cross from
+ * the QKV call to attention as e4m3 codes with one static scale each,
+ *   s_q = fp32(sqrt(128) * max|qn_w|) / 448 (fp32 arithmetic, sqrt(128) as
+ *   the fp32 constant 11.3137085), code = e4m3(fp32(q * fp32(1 / s_q)))
+ * written as 448 / fp32(11.3137085 * max|qn_w|), and likewise for k with
+ * kn_w.  RMSNorm then RoPE bound every element of a head row by
+ * sqrt(128) max|w|, so no code saturates; S = s_q s_k (Q8 K8^T).
+ * Code matrices are row-major bytes; every row length is a multiple of 16
+ * bytes as for the bf16 calls (D % 64, I, F % 128). */
 typedef uint8_t h3_e4m3;
 
 /* Row quantisation of a bf16 matrix (weights offline; activations between
@@ -313,7 +328,9 @@ int h3_adaln_norm_modulate_e4m3(const h3_dims* dims, const h3_ranges* ranges, co
 
 /* A4 + A5 from e4m3 operands: as h3_qkv_qknorm_mrope with xm = (xq, xs)
  * [L_pad][D] and Wqkv = (Wq, Ws) [3I][D], Ws per output channel.  q, k, v
- * bf16 head-major [H][L_pad][128]. */
+ * bf16 head-major [H][L_pad][128]; with flags & H3_QK_E4M3, q and k receive
+ * e4m3 codes instead, [H][L_pad][128] bytes (the buffers may be the bf16
+ * ones: half of each is used), v stays bf16. */
 int h3_qkv_qknorm_mrope_e4m3(const h3_dims* dims, const h3_ranges* ranges, const h3_e4m3* xq, const float* xs,
                              const h3_e4m3* Wq, const float* Ws, const h3_bf16* qn_w, const h3_bf16* kn_w,
                              const float* pos, int flags, h3_bf16* q, h3_bf16* k, h3_bf16* v, void* stream);
@@ -360,8 +377,9 @@ typedef struct h3_block_buffers_e4m3 {
 } h3_block_buffers_e4m3;
 
 /* One whole block with e4m3 GEMMs: h3_adaln_norm_modulate_e4m3 (MSA),
- * h3_qkv_qknorm_mrope_e4m3, h3_attention (bf16), h3_quantize_rows_e4m3 of o,
- * h3_gated_residual_e4m3, h3_adaln_norm_modulate_e4m3 (MLP),
+ * h3_qkv_qknorm_mrope_e4m3, h3_attention (bf16, or e4m3 Q K^T with
+ * flags & H3_QK_E4M3: buf->q, buf->k then hold codes), h3_quantize_rows_e4m3
+ * of o, h3_gated_residual_e4m3, h3_adaln_norm_modulate_e4m3 (MLP),
  * h3_ffn_swiglu_e4m3.  Nothing is launched if any argument is invalid. */
 int h3_block_forward_e4m3(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod,
                           const float* pos, const h3_block_weights_e4m3* w, const h3_block_buffers_e4m3* buf,

@@ -43,11 +43,16 @@ constexpr int NUM_THREADS = 320;
 constexpr int TILE = 128;
 constexpr int HALF_BYTES = TILE * 64 * 2;   // 128 rows x 64 bf16 = 16 KB
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 32 KB
-constexpr int SMEM_Q = 0;                   // 2 query tiles
-constexpr int SMEM_K = SMEM_Q + 2 * TILE_BYTES;  // 2 stages
-constexpr int SMEM_V = SMEM_K + 2 * TILE_BYTES;  // 2 stages
-constexpr int SMEM_BAR = SMEM_V + 2 * TILE_BYTES;
-constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
+// Q and K tiles: bf16 (32 KB, two 64-column halves) or, with QK8, e4m3 codes
+// (16 KB, one 128-byte row per token)
+template <bool QK8> struct Layout {
+  static constexpr int QK_TILE = QK8 ? TILE * 128 : TILE_BYTES;
+  static constexpr int Q = 0;                  // 2 query tiles
+  static constexpr int K = Q + 2 * QK_TILE;    // 2 stages
+  static constexpr int V = K + 2 * QK_TILE;    // 2 stages
+  static constexpr int BAR = V + 2 * TILE_BYTES;
+  static constexpr int BYTES = BAR + 256 + 1024;
+};
 constexpr int TMEM_COLS = 512;
 // A 64-key half whose exponentials (against the current reference) sum past
 // this moves the reference: every p of an accepted half is <= 2^16, so p, the
@@ -76,17 +81,23 @@ struct AttnOut {
   bf16* shard[8];
 };
 
+// QK8: Q and K are e4m3 codes of q * 448 / (sqrt(128) max|qn_w|) and of
+// k * 448 / (sqrt(128) max|kn_w|); S = Q K^T is taken with kind::f8f6f4 MMAs
+// and the two scales folded into the softmax scale.  P V stays bf16.
+template <bool QK8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnOut out, int H, int L,
-                        int L_pad, float scale_log2) {
+                        int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w) {
+  using LY = Layout<QK8>;
+  constexpr int QK_TILE = LY::QK_TILE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = smem + SMEM_Q;
-  uint8_t* sK = smem + SMEM_K;
-  uint8_t* sV = smem + SMEM_V;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);
+  uint8_t* sQ = smem + LY::Q;
+  uint8_t* sK = smem + LY::K;
+  uint8_t* sV = smem + LY::V;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2] per K stage
   uint64_t* v_full = bars + 3;    // [2] per V stage
@@ -98,6 +109,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* drain = bars + 17;    // the MMA issuer's last commit before teardown
   uint64_t* pv0_done = bars + 18; // [2] per query tile: PV on the first key half complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  float* qk_scale = reinterpret_cast<float*>(bars + 21);  // QK8: dequantisation of S
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -130,6 +142,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
+  if (QK8 && warp == 2) {
+    // (sqrt(128) max|qn_w| / 448) (sqrt(128) max|kn_w| / 448)
+    float mq = 0.f, mk = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mq = fmaxf(mq, fabsf(__bfloat162float(qn_w[lane * 4 + i])));
+      mk = fmaxf(mk, fabsf(__bfloat162float(kn_w[lane * 4 + i])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+      mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+    }
+    if (lane == 0) *qk_scale = ((11.3137085f * mq) / 448.0f) * ((11.3137085f * mk) / 448.0f);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -137,20 +164,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
-      tma_load_2d(sQ, &tmQ, q_full, 0, row0 + qt0 * TILE);
-      tma_load_2d(sQ + HALF_BYTES, &tmQ, q_full, 64, row0 + qt0 * TILE);
-      tma_load_2d(sQ + TILE_BYTES, &tmQ, q_full, 0, row0 + qt1 * TILE);
-      tma_load_2d(sQ + TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, row0 + qt1 * TILE);
+      mbar_arrive_expect_tx(q_full, 2 * QK_TILE);
+      if (QK8) {
+        tma_load_2d(sQ, &tmQ, q_full, 0, row0 + qt0 * TILE);
+        tma_load_2d(sQ + QK_TILE, &tmQ, q_full, 0, row0 + qt1 * TILE);
+      } else {
+        tma_load_2d(sQ, &tmQ, q_full, 0, row0 + qt0 * TILE);
+        tma_load_2d(sQ + HALF_BYTES, &tmQ, q_full, 64, row0 + qt0 * TILE);
+        tma_load_2d(sQ + TILE_BYTES, &tmQ, q_full, 0, row0 + qt1 * TILE);
+        tma_load_2d(sQ + TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, row0 + qt1 * TILE);
+      }
       long long k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
-        uint8_t* dk = sK + st * TILE_BYTES;
+        uint8_t* dk = sK + st * QK_TILE;
         uint8_t* dv = sV + st * TILE_BYTES;
         if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) break;
-        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
+        mbar_arrive_expect_tx(&k_full[st], QK_TILE);
         tma_load_2d(dk, &tmK, &k_full[st], 0, row0 + j * TILE);
-        tma_load_2d(dk + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
+        if (!QK8) tma_load_2d(dk + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
         ++k_issued;
         if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
@@ -166,6 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // The whole warp runs the issue loop, converged; one elected lane issues.
     const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+    const uint32_t idesc_s8 = idesc_e4m3_f32(128, 128);
     const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);  // V is MN-major (d contiguous)
     // Shared-memory descriptors are computed once; an MMA then costs one
     // 64-bit add (the start-address field is bits [0,14) in 16-byte units,
@@ -175,12 +208,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint64_t v_desc = sdesc_sw128(smem_u32(sV), HALF_BYTES, 1024);
     // S_t = Q_t K_j^T into TMEM columns [256t, 256t + 128)
     auto issue_s = [&](int t, int j) {
-      const uint64_t qd = q_desc + (uint64_t)((t * TILE_BYTES) >> 4);
-      const uint64_t kd = k_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
+      const uint64_t qd = q_desc + (uint64_t)((t * QK_TILE) >> 4);
+      const uint64_t kd = k_desc + (uint64_t)(((j & 1) * QK_TILE) >> 4);
+      if constexpr (QK8) {
+        // one 128-byte row per token: four MMAs of K = 32 codes (32 bytes)
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-        umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          umma_e4m3(tmem + t * 256, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), idesc_s8, kk != 0 ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+          umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+        }
       }
       umma_commit(&s_full[t]);
     };
@@ -231,6 +271,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     drain_mmas(drain);
   } else {
     const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    // log2(e) / sqrt(128), times the dequantisation of e4m3 S
+    const float sl2 = QK8 ? scale_log2 * *qk_scale : scale_log2;
     const int qw = warp & 3;        // TMEM lane quarter this warp may access
     const int r = qw * 32 + lane;   // query row inside the tile
     const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
@@ -272,9 +314,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // that half's row max, with O and the sums rescaled first.  A half that
       // passed the check lies within 2^16 of the reference, so it stays in
       // range when the reference moves up.  No per-tile row max otherwise.
-      if (j == 0) m_ref = row_max(0, 128) * scale_log2;
-      const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
-      // p = 2^(s * scale_log2 - m_ref) on the MUFU unit (masked keys, -inf,
+      if (j == 0) m_ref = row_max(0, 128) * sl2;
+      const uint64_t sc2 = f2_pack(sl2, sl2);
+      // p = 2^(s * sl2 - m_ref) on the MUFU unit (masked keys, -inf,
       // give exactly 0); returns this row's sum over the half
       auto exp_half = [&](int hf, uint32_t* pk) {
         const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
@@ -311,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = hf * 64; c < hf * 64 + 64; ++c)
               if (c >= valid) s[c] = -INFINITY;
           }
-          const float m_new = fmaxf(m_ref, row_max(hf * 64, 64) * scale_log2);
+          const float m_new = fmaxf(m_ref, row_max(hf * 64, 64) * sl2);
           const float a = ex2_approx(m_ref - m_new);  // 1 where the reference holds
           m_ref = m_new;
           // O must hold every PV issued against the old reference before it
@@ -384,16 +426,26 @@ using namespace attn_detail;
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
                     uint32_t box_rows);
+bool make_tmap_e4m3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                    uint32_t box_rows);
 
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
-  static unsigned long long attr_done = 0;
-  cudaError_t aerr =
-      ensure_smem_attr(reinterpret_cast<const void*>(attention_tc_kernel), attn_detail::SMEM_BYTES, &attr_done);
+  const bool qk8 = p.qk8 != 0;
+  if (qk8 && (p.qn_w == nullptr || p.kn_w == nullptr)) return cudaErrorInvalidValue;
+  static unsigned long long attr_done[2] = {0, 0};
+  const void* kfn = qk8 ? reinterpret_cast<const void*>(attention_tc_kernel<true>)
+                        : reinterpret_cast<const void*>(attention_tc_kernel<false>);
+  cudaError_t aerr = ensure_smem_attr(kfn, qk8 ? Layout<true>::BYTES : Layout<false>::BYTES, &attr_done[qk8 ? 1 : 0]);
   if (aerr != cudaSuccess) return aerr;
   CUtensorMap tq, tk, tv;
   const uint64_t rows = (uint64_t)p.H * p.L_pad;
-  if (!make_tmap_bf16(&tq, p.q, rows, 128, 128, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16(&tk, p.k, rows, 128, 128, 128)) return cudaErrorInvalidValue;
+  if (qk8) {
+    if (!make_tmap_e4m3(&tq, p.q, rows, 128, 128, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_e4m3(&tk, p.k, rows, 128, 128, 128)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_tmap_bf16(&tq, p.q, rows, 128, 128, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tk, p.k, rows, 128, 128, 128)) return cudaErrorInvalidValue;
+  }
   if (!make_tmap_bf16(&tv, p.v, rows, 128, 128, 128)) return cudaErrorInvalidValue;
   const int n_qt = p.L_pad / attn_detail::TILE;
   AttnOut out;
@@ -411,8 +463,12 @@ cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
     out.shard[0] = p.o;
   }
   dim3 grid((n_qt + 1) / 2, p.H);
-  attention_tc_kernel<<<grid, attn_detail::NUM_THREADS, attn_detail::SMEM_BYTES, stream>>>(
-      tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2);
+  if (qk8)
+    attention_tc_kernel<true><<<grid, attn_detail::NUM_THREADS, Layout<true>::BYTES, stream>>>(
+        tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, p.qn_w, p.kn_w);
+  else
+    attention_tc_kernel<false><<<grid, attn_detail::NUM_THREADS, Layout<false>::BYTES, stream>>>(
+        tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, nullptr, nullptr);
   return cudaGetLastError();
 }
 

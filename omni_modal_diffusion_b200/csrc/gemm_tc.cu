@@ -187,6 +187,28 @@ __device__ __forceinline__ void epi_swiglu(const GemmEpilogue& e, uint32_t tb, i
   }
 }
 
+// One warp: the e4m3 code scales of q and k, 448 / (sqrt(128) max|w|) for
+// the norm weights w = qn_w, kn_w (RMSNorm then RoPE bound every element of
+// a head row by sqrt(128) max|w|, so no code saturates).
+__device__ __forceinline__ void qk_e4m3_inv_scales(const GemmEpilogue& e, float* qk_inv) {
+  const int lane = threadIdx.x & 31;
+  float mq = 0.f, mk = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mq = fmaxf(mq, fabsf(__bfloat162float(e.qn_w[lane * 4 + i])));
+    mk = fmaxf(mk, fabsf(__bfloat162float(e.kn_w[lane * 4 + i])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+    mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+  }
+  if (lane == 0) {
+    qk_inv[0] = 448.0f / (11.3137085f * mq);
+    qk_inv[1] = 448.0f / (11.3137085f * mk);
+  }
+}
+
 // sin and cos of a RoPE angle on the MUFU unit.  The angle is first reduced
 // to [-pi, pi] with 2 pi split into its nearest fp32 value H = 6.28318548...
 // and the remainder T = 2 pi - H = -1.7484556e-7 (two-term Cody-Waite
@@ -206,7 +228,8 @@ __device__ __forceinline__ void rope_sincos(float a, float* s, float* c) {
 // TMEM per head: the sum of squares of the 128 values, then chunk by chunk
 // normalise, rotate and store (no 128-value array in registers).
 __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int m, int n0, const float* freq,
-                                        const uint8_t* axis_of_pair, int h_lo = 0, int h_hi = 2) {
+                                        const uint8_t* axis_of_pair, const float* qk_inv, int h_lo = 0,
+                                        int h_hi = 2) {
   float p3[3] = {0.f, 0.f, 0.f};
   if (m < e.L_pad) {
     p3[0] = e.pos[(long)m * 3 + 0];
@@ -272,7 +295,18 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
           v[2 * i + 1] = a * sn + bb * cs;
         }
       }
-      if (dst) {
+      if (dst && part < 2 && e.qk_e4m3) {
+        // e4m3 codes of v * 448 / (sqrt(128) max|w|): 32 bytes of the head's
+        // 128-byte row
+        const float inv = qk_inv[part];
+        uint32_t w4[8];
+#pragma unroll
+        for (int d = 0; d < 32; d += 4)
+          w4[d / 4] = cvt_e4m3x2(v[d] * inv, v[d + 1] * inv) | (cvt_e4m3x2(v[d + 2] * inv, v[d + 3] * inv) << 16);
+        uint8_t* dst8 = reinterpret_cast<uint8_t*>(part == 0 ? e.q : e.k) + ((long)h * e.L_pad + m) * 128 + c * 32;
+        reinterpret_cast<uint4*>(dst8)[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        reinterpret_cast<uint4*>(dst8)[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
+      } else if (dst) {
 #pragma unroll
         for (int d = 0; d < 32; d += 8) {
           uint4 o;
@@ -329,6 +363,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
+  float* qk_inv = reinterpret_cast<float*>(axis_of_pair + 64);
   float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + MISC_BYTES);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -364,6 +399,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     freq[i] = powf(e.theta, -2.0f * (float)i_sec / (float)d_sec);
     axis_of_pair[i] = (uint8_t)ax;
   }
+  if (e.mode == EPI_QKV && e.qk_e4m3 && threadIdx.x >= 128 && threadIdx.x < 160) qk_e4m3_inv_scales(e, qk_inv);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -450,7 +486,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         case EPI_STORE_F32: epi_store_f32(e, tb, m, nt * BN, epi_stage + q * 32 * EPI_PITCH); break;
         case EPI_GATED_RESID: epi_gated_resid(e, tb, m, nt * BN); break;
         case EPI_SWIGLU: epi_swiglu(e, tb, m, nt); break;
-        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair); break;
+        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair, qk_inv); break;
         case EPI_UNPATCH: epi_unpatch(e, tb, m, nt * BN); break;
         default: break;
       }
@@ -510,6 +546,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   float* freq = reinterpret_cast<float*>(tmem_slot + 4);
   uint8_t* axis_of_pair = reinterpret_cast<uint8_t*>(freq + 64);
+  float* qk_inv = reinterpret_cast<float*>(axis_of_pair + 64);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
@@ -545,6 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
     freq[i] = powf(e.theta, -2.0f * (float)i_sec / (float)d_sec);
     axis_of_pair[i] = (uint8_t)ax;
   }
+  if (e.mode == EPI_QKV && e.qk_e4m3 && threadIdx.x >= 128 && threadIdx.x < 160) qk_e4m3_inv_scales(e, qk_inv);
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // barriers of both CTAs initialised before any remote arrival
@@ -650,7 +688,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_NUM_THREADS, 1)
             epi_gated_resid(e, tb, m, nt * BN);
           break;
         case EPI_SWIGLU: epi_swiglu(e, tb, m, nt, sub * 2, sub * 2 + 2); break;
-        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair, sub, sub + 1); break;
+        case EPI_QKV: epi_qkv(e, tb, m, nt * BN, freq, axis_of_pair, qk_inv, sub, sub + 1); break;
         default: break;
       }
       tc_fence_before();
@@ -708,8 +746,8 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   return make_tmap_128b(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, rows, cols, row_stride_elems, box_rows);
 }
 
-static bool make_tmap_e4m3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                           uint64_t row_stride_elems, uint32_t box_rows) {
+bool make_tmap_e4m3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                    uint32_t box_rows) {
   return make_tmap_128b(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, rows, cols, row_stride_elems, box_rows);
 }
 

@@ -289,6 +289,8 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
   H3_CHECK(check_ranges(ranges, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
     return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  if (flags & ~H3_QK_NORM_ROPE_IN_QKV)
+    return fail(H3_ERR_UNSUPPORTED, "%s: e4m3 q/k output needs h3_qkv_qknorm_mrope_e4m3", __func__);
   H3_REQUIRE_PTR(xm);
   H3_REQUIRE_PTR(Wqkv);
   H3_REQUIRE_PTR(qn_w);
@@ -307,19 +309,25 @@ int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q,
                  const h3_bf16* v, const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
                  h3_bf16* o, void* stream) {
   H3_TRACE();
-  (void)qn_w;
-  (void)kn_w;
   (void)pos;
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
     return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  if (flags & ~(H3_QK_NORM_ROPE_IN_QKV | H3_QK_E4M3)) return fail(H3_ERR_UNSUPPORTED, "%s: unknown flags", __func__);
   H3_REQUIRE_PTR(q);
   H3_REQUIRE_PTR(k);
   H3_REQUIRE_PTR(v);
   H3_REQUIRE_PTR(o);
   AttnProblem p;
   memset(&p, 0, sizeof(p));
+  if (flags & H3_QK_E4M3) {  // q, k: e4m3 codes whose scales follow from qn_w, kn_w
+    H3_REQUIRE_PTR(qn_w);
+    H3_REQUIRE_PTR(kn_w);
+    p.qk8 = 1;
+    p.qn_w = reinterpret_cast<const bf16*>(qn_w);
+    p.kn_w = reinterpret_cast<const bf16*>(kn_w);
+  }
   p.q = reinterpret_cast<const bf16*>(q);
   p.k = reinterpret_cast<const bf16*>(k);
   p.v = reinterpret_cast<const bf16*>(v);

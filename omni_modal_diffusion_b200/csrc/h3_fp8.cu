@@ -88,7 +88,9 @@ int h3_qkv_qknorm_mrope_e4m3(const h3_dims* dims, const h3_ranges* ranges, const
   H3_REQUIRE_PTR(q);
   H3_REQUIRE_PTR(k);
   H3_REQUIRE_PTR(v);
+  if (flags & ~(H3_QK_NORM_ROPE_IN_QKV | H3_QK_E4M3)) return fail(H3_ERR_UNSUPPORTED, "%s: unknown flags", __func__);
   GemmProblem p = with_e4m3(qkv_problem(dims, ranges, xq, Wq, qn_w, kn_w, pos, q, k, v), xs, Ws);
+  p.epi.qk_e4m3 = (flags & H3_QK_E4M3) ? 1 : 0;
   cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_qkv_qknorm_mrope_e4m3");
   return ok();

@@ -39,6 +39,10 @@ struct GemmEpilogue {
   int L_pad, I;
   int rope_t, rope_h, rope_w;
   float theta, eps_qk;
+  // EPI_QKV with qk_e4m3: q and k are written as e4m3 codes (q, k then point
+  // to [H][L_pad][128] bytes) of value * 448 / (sqrt(128) max|w|), w the
+  // head's norm weight; v stays bf16
+  int qk_e4m3;
   // EPI_UNPATCH: token grid (T, Ht, Wt), latent channels
   int Ht, Wt, C_lat;
   // e4m3 operands: acc[m][n] *= a_scale[m] * b_scale[n] before the epilogue
@@ -92,6 +96,11 @@ struct AttnProblem {
   int sp_n, sp_L_shard, sp_head0;
   long sp_ld;
   bf16* sp_o[8];
+  // qk8: q, k hold e4m3 codes (one byte per element) written by the QKV
+  // epilogue with qk_e4m3; qn_w, kn_w give their scales
+  int qk8;
+  const bf16* qn_w;
+  const bf16* kn_w;
 };
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream);
 

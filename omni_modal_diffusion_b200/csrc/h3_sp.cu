@@ -94,6 +94,8 @@ int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3
     return fail(H3_ERR_SHAPE, "%s: shard L_pad (%d) != layout L_shard (%d)", __func__, shard->L_pad, layout->L_shard);
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
     return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  if (flags & ~H3_QK_NORM_ROPE_IN_QKV)
+    return fail(H3_ERR_UNSUPPORTED, "%s: only H3_QK_NORM_ROPE_IN_QKV (e4m3 q/k are not sequence parallel)", __func__);
   H3_REQUIRE_PTR(xm);
   H3_REQUIRE_PTR(Wqkv);
   H3_REQUIRE_PTR(qn_w);
@@ -123,6 +125,8 @@ int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp
   H3_CHECK(check_layout(dims, layout, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
     return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  if (flags & ~H3_QK_NORM_ROPE_IN_QKV)
+    return fail(H3_ERR_UNSUPPORTED, "%s: only H3_QK_NORM_ROPE_IN_QKV (e4m3 q/k are not sequence parallel)", __func__);
   H3_CHECK(check_peers(peers, layout->n_ranks, false, true, __func__));
   const int r = layout->rank;
   if (!peers->q[r] || !peers->k[r] || !peers->v[r])

@@ -19,6 +19,7 @@ H3_OK, H3_ERR_NULL, H3_ERR_SHAPE, H3_ERR_ALIGN, H3_ERR_UNSUPPORTED, H3_ERR_CUDA,
 H3_TEXT, H3_AUDIO, H3_VIDEO = 0, 1, 2
 H3_MSA, H3_MLP = 0, 1
 H3_QK_NORM_ROPE_IN_QKV = 1
+H3_QK_E4M3 = 2  # q, k as e4m3 codes between the e4m3 QKV call and attention
 
 EXPORTS = (
     "h3_last_error", "h3_version", "h3_make_ranges", "h3_sigma_schedule", "h3_embed_pack",
@@ -204,7 +205,8 @@ def h3_qkv_qknorm_mrope(dims, ranges, xm, Wqkv, qn_w, kn_w, pos, q, k, v, flags=
 
 
 def h3_attention(dims, ranges, q, k, v, o, qn_w=None, kn_w=None, pos=None, flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
-    _check(lib().h3_attention(ctypes.byref(dims), ctypes.byref(ranges), _ptr(q, BF16, "q"), _ptr(k, BF16, "k"),
+    qk = U8 if flags & H3_QK_E4M3 else BF16
+    _check(lib().h3_attention(ctypes.byref(dims), ctypes.byref(ranges), _ptr(q, qk, "q"), _ptr(k, qk, "k"),
                               _ptr(v, BF16, "v"), _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"),
                               _ptr(pos, F32, "pos"), flags, _ptr(o, BF16, "o"), _stream(stream)))
 
@@ -313,7 +315,8 @@ def h3_qkv_qknorm_mrope_e4m3(dims, ranges, xq, xs, Wq, Ws, qn_w, kn_w, pos, q, k
     _check(lib().h3_qkv_qknorm_mrope_e4m3(ctypes.byref(dims), ctypes.byref(ranges), _ptr(xq, U8, "xq"),
                                           _ptr(xs, F32, "xs"), _ptr(Wq, U8, "Wq"), _ptr(Ws, F32, "Ws"),
                                           _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"), _ptr(pos, F32, "pos"),
-                                          flags, _ptr(q, BF16, "q"), _ptr(k, BF16, "k"), _ptr(v, BF16, "v"),
+                                          flags, _ptr(q, U8 if flags & H3_QK_E4M3 else BF16, "q"),
+                                          _ptr(k, U8 if flags & H3_QK_E4M3 else BF16, "k"), _ptr(v, BF16, "v"),
                                           _stream(stream)))
 
 
@@ -342,7 +345,12 @@ def block_weights_e4m3(W: dict) -> BlockWeightsE4m3:
 
 
 def block_buffers_e4m3(B: dict) -> BlockBuffersE4m3:
-    dt = {"xq": U8, "xs": F32, "q": BF16, "k": BF16, "v": BF16, "o": BF16, "oq": U8, "os": F32, "ws": U8}
+    """q and k may be bf16 or, for the H3_QK_E4M3 block, uint8 code buffers."""
+    dt = {"xq": U8, "xs": F32, "q": (BF16, U8), "k": (BF16, U8), "v": BF16, "o": BF16, "oq": U8, "os": F32, "ws": U8}
+    for n in ("q", "k"):
+        if B[n].dtype not in dt[n]:
+            raise TypeError(f"{n} must be bfloat16 or uint8, got {B[n].dtype}")
+        dt[n] = B[n].dtype
     return BlockBuffersE4m3(*(_ptr(B[n], dt[n], n) for n in E4M3_BUFFER_FIELDS))
 
 

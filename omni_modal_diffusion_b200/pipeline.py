@@ -100,15 +100,21 @@ class H3BlockStep:
         self.oq = torch.empty(Lp, I, dtype=torch.uint8, device=dev)
         self.os = torch.empty(Lp, dtype=torch.float32, device=dev)
         self.ws8 = torch.empty(h3.h3_ffn_e4m3_workspace_bytes(self.dims, Lp), dtype=torch.uint8, device=dev)
+        # q, k as e4m3 codes (H3_QK_E4M3)
+        self.q8 = torch.empty(self.w.H, Lp, 128, dtype=torch.uint8, device=dev)
+        self.k8 = torch.empty(self.w.H, Lp, 128, dtype=torch.uint8, device=dev)
 
-    def block_e4m3(self, mod, W8: dict, stream=None):
+    def block_e4m3(self, mod, W8: dict, stream=None, qk_e4m3: bool = False):
         """One block over self.x with the four GEMMs in e4m3 (W8 from
-        quantize_block_weights_e4m3; alloc_e4m3 called once before)."""
+        quantize_block_weights_e4m3; alloc_e4m3 called once before);
+        qk_e4m3 also passes q, k to attention as e4m3 codes (H3_QK_E4M3)."""
         d, r = self.dims, self.ranges
+        flags = h3.H3_QK_NORM_ROPE_IN_QKV | (h3.H3_QK_E4M3 if qk_e4m3 else 0)
+        q, k = (self.q8, self.k8) if qk_e4m3 else (self.q, self.k)
         h3.h3_adaln_norm_modulate_e4m3(d, r, self.x, mod, h3.H3_MSA, self.xq, self.xs, stream=stream)
         h3.h3_qkv_qknorm_mrope_e4m3(d, r, self.xq, self.xs, W8["Wqkv"], W8["Wqkv_s"], W8["qn_w"], W8["kn_w"],
-                                    self.pos, self.q, self.k, self.v, stream=stream)
-        h3.h3_attention(d, r, self.q, self.k, self.v, self.o, stream=stream)
+                                    self.pos, q, k, self.v, flags=flags, stream=stream)
+        h3.h3_attention(d, r, q, k, self.v, self.o, qn_w=W8["qn_w"], kn_w=W8["kn_w"], flags=flags, stream=stream)
         h3.h3_quantize_rows_e4m3(self.o, self.oq, self.os, stream=stream)
         h3.h3_gated_residual_e4m3(d, r, self.x, self.oq, self.os, W8["Wo"], W8["Wo_s"], mod, h3.H3_MSA,
                                   stream=stream)
@@ -157,20 +163,25 @@ class H3Sampler:
     e4m3=True runs the blocks with their four GEMMs on e4m3 operands
     (h3_block_forward_e4m3): each block's weights are quantised once on the
     GPU here and only the e4m3 copies are kept (the caller may drop its bf16
-    block weights afterwards)."""
+    block weights afterwards).  qk_e4m3=True (with e4m3) also takes attention's
+    Q K^T on e4m3 codes (H3_QK_E4M3)."""
 
     def __init__(self, w: Workload, io_weights: dict, block_weights: list, device="cuda",
-                 shift_video: float = 12.0, shift_audio: float = 3.0, e4m3: bool = False):
+                 shift_video: float = 12.0, shift_audio: float = 3.0, e4m3: bool = False, qk_e4m3: bool = False):
+        if qk_e4m3 and not e4m3:
+            raise ValueError("qk_e4m3 needs e4m3")
         self.st = H3BlockStep(w, device=device, weights=io_weights)
         st = self.st
         self.e4m3 = e4m3
+        self.flags = h3.H3_QK_NORM_ROPE_IN_QKV | (h3.H3_QK_E4M3 if qk_e4m3 else 0)
         if e4m3:
             st.alloc_e4m3()
             self.block_tensors = [st.quantize_block_weights_e4m3(Wb) for Wb in block_weights]
             torch.cuda.synchronize(st.device)
             self.blocks = [h3.block_weights_e4m3(Wb) for Wb in self.block_tensors]
-            self.bufs = h3.block_buffers_e4m3({"xq": st.xq, "xs": st.xs, "q": st.q, "k": st.k, "v": st.v,
-                                               "o": st.o, "oq": st.oq, "os": st.os, "ws": st.ws8})
+            self.bufs = h3.block_buffers_e4m3({"xq": st.xq, "xs": st.xs, "q": st.q8 if qk_e4m3 else st.q,
+                                               "k": st.k8 if qk_e4m3 else st.k, "v": st.v, "o": st.o, "oq": st.oq,
+                                               "os": st.os, "ws": st.ws8})
         else:
             self.block_tensors = block_weights            # keep the tensors alive
             self.blocks = [h3.block_weights(Wb) for Wb in block_weights]
@@ -186,7 +197,8 @@ class H3Sampler:
         st.embed(text, video_bf16, audio_bf16, stream)
         forward = h3.h3_block_forward_e4m3 if self.e4m3 else h3.h3_block_forward
         for b in range(self.n_layers):
-            forward(st.dims, st.ranges, st.x, mod_all[s, b], st.pos, self.blocks[b], self.bufs, stream=stream)
+            forward(st.dims, st.ranges, st.x, mod_all[s, b], st.pos, self.blocks[b], self.bufs, flags=self.flags,
+                    stream=stream)
         st.head(stream)
         h3.h3_euler_step_bf16(lat_video, st.v_video, sv[s], sv[s + 1], video_bf16, stream=stream)
         h3.h3_euler_step_bf16(lat_audio, st.v_audio, sa[s], sa[s + 1], audio_bf16, stream=stream)

@@ -24,6 +24,13 @@ they fix no format.  This module states the scheme the FP8 path computes:
     (row of the [out, in] weight), and an FP8 GEMM is
     out[m, n] = scale_a[m] * scale_b[n] * sum_k dec(qa[m, k]) dec(qb[n, k]),
     after which the bf16 path's epilogues apply unchanged.
+  * Optionally (H3_QK_E4M3) q and k reach attention as e4m3 codes with one
+    static scale each, taken from the bound that RMSNorm then RoPE put on a
+    head row: every element is at most sqrt(128) max|w| in magnitude (w the
+    norm weight), so s = fp32(fp32(sqrt(128) * max|w|) / 448) and
+    code = e4m3(fp32(x * fp32(448 / fp32(sqrt(128) * max|w|)))), in fp32
+    arithmetic with sqrt(128) as the fp32 constant 11.3137085.  Attention
+    then sees S = s_q s_k sum dec(q) dec(k).
 
 Parity pins (tests/test_oracle_fp8_pins.py): the value table against the
 closed form of every code; encoding against a brute-force nearest search and
@@ -139,6 +146,29 @@ def quantize_weight(W) -> tuple[np.ndarray, np.ndarray]:
     return quantize_rows(W)
 
 
+QK_SQRT128 = np.float32(11.3137085)
+
+
+def qk_code_scale(w) -> tuple[np.float32, np.float32]:
+    """(inverse scale, scale) of the e4m3 codes of q or k rows normalised
+    with weight w (see the module docstring), in fp32."""
+    m = np.float32(np.max(np.abs(np.asarray(w, np.float32))))
+    d = np.float32(QK_SQRT128 * m)
+    return np.float32(np.float32(448.0) / d), np.float32(d / np.float32(448.0))
+
+
+def quantize_qk(x, w) -> np.ndarray:
+    """e4m3 codes of x (q or k rows after RMSNorm with weight w and RoPE):
+    e4m3(fp32(x * inv))."""
+    inv, _ = qk_code_scale(w)
+    return e4m3_encode((np.asarray(x, np.float64) * np.float64(inv)).astype(np.float32))
+
+
+def dequantize_qk(codes, w) -> np.ndarray:
+    _, s = qk_code_scale(w)
+    return e4m3_decode(codes) * np.float64(s)
+
+
 def qkv_qknorm_mrope_e4m3(xq, xs, Wq, Ws, qn_w, kn_w, pos, n_heads, head_dim=128, split=(32, 48, 48)):
     """QKV from e4m3 operands, then the bf16 path's per-head Q/K RMSNorm and
     3-D RoPE on the fp32 accumulator."""
@@ -164,15 +194,19 @@ def ffn_down_e4m3(x, hq, hs, Wdq, Wds, mod, ranges, rows=None):
 
 
 def block_forward_e4m3(x, mod, ranges, pos, Wqkv_q, Wqkv_s, qn_w, kn_w, Wo_q, Wo_s, Wgu_q, Wgu_s, Wd_q, Wd_s,
-                       n_heads, head_dim=128, split=(32, 48, 48), return_parts=False):
+                       n_heads, head_dim=128, split=(32, 48, 48), return_parts=False, qk_e4m3=False):
     """The block with its four GEMMs in e4m3.  Quantisation points: the two
     modulated LayerNorm outputs (from their fp32 values), the attention
     output and the SwiGLU hidden state (from the bf16 tensors the path
-    stores).  Attention itself stays in the bf16 path's form."""
+    stores), and with qk_e4m3 q and k (static scales, from their fp32
+    values).  Attention itself stays in the bf16 path's form."""
     x = np.asarray(x, np.float64)
     xm1 = O.adaln_modulate(x, mod, ranges, O.MSA)
     xq1, xs1 = quantize_rows(xm1)
     q, k, v = qkv_qknorm_mrope_e4m3(xq1, xs1, Wqkv_q, Wqkv_s, qn_w, kn_w, pos, n_heads, head_dim, split)
+    if qk_e4m3:
+        q = dequantize_qk(quantize_qk(q, qn_w), qn_w)
+        k = dequantize_qk(quantize_qk(k, kn_w), kn_w)
     o = O.attention(q, k, v)
     oq, os_ = quantize_rows(O.round_to_bf16(o))
     x1 = gated_residual_e4m3(x, oq, os_, Wo_q, Wo_s, mod, ranges)

@@ -111,3 +111,38 @@ def test_gemm_triple_loop():
             for k in range(7):
                 acc += F.e4m3_value(int(qa[m, k])) * F.e4m3_value(int(qb[n, k]))
             assert out[m, n] == pytest.approx(float(sa[m]) * float(sb[n]) * acc, rel=1e-12, abs=1e-300)
+
+
+def test_qk_codes_static_scale():
+    """q / k codes with the static scale from the norm weight: the scale is
+    fp32(sqrt(128) max|w|) / 448; the bound that RMSNorm then RoPE give a head
+    row (every element at most sqrt(128) max|w|) lands on the largest code
+    without passing it; every finite code of the scale's grid round-trips;
+    and dequantised values are within half a step of a 3-bit mantissa."""
+    rng = np.random.default_rng(11)
+    w = (1 + 0.1 * rng.standard_normal(128)).astype(np.float32)
+    w[17] = -1.6  # the bound uses |w|
+    inv, s = F.qk_code_scale(w)
+    assert s == np.float32(np.float32(np.float32(11.3137085) * np.float32(1.6)) / np.float32(448.0))
+    assert abs(float(inv) * float(s) - 1.0) < 1e-6
+    # extreme row: all of the row's energy in one element, |x| = sqrt(128) max|w|
+    x = np.zeros((1, 128))
+    x[0, 5] = -np.sqrt(128.0) * 1.6
+    c = F.quantize_qk(x, w)
+    assert c[0, 5] == 0xFE                       # -448
+    # rows that RMSNorm (weight w) and a rotation of pairs produce stay within the bound
+    r = rng.standard_normal((256, 128))
+    r = r / np.sqrt((r ** 2).mean(1, keepdims=True)) * w.astype(np.float64)
+    ang = rng.uniform(-np.pi, np.pi, (256, 64))
+    a, b = r[:, 0::2], r[:, 1::2]
+    rot = np.empty_like(r)
+    rot[:, 0::2], rot[:, 1::2] = a * np.cos(ang) - b * np.sin(ang), a * np.sin(ang) + b * np.cos(ang)
+    assert np.all(np.abs(rot) <= np.sqrt(128.0) * 1.6 + 1e-12)
+    dec = F.dequantize_qk(F.quantize_qk(rot, w), w)
+    assert np.all(np.abs(F.e4m3_decode(F.quantize_qk(rot, w))) <= 448.0)
+    err = np.abs(dec - rot)
+    assert np.all(err <= np.maximum(np.abs(rot) * 2.0 ** -4, 2.0 ** -10 * float(s)) * (1 + 1e-6) + 1e-7)
+    # every finite code of the grid round-trips exactly
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    vals = F.e4m3_decode(codes) * np.float64(s)
+    assert np.array_equal(F.quantize_qk(vals, w) & 0x7F, codes & 0x7F)
