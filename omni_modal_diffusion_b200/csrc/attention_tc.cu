@@ -21,6 +21,9 @@
 //              O / l to global memory.
 // TMEM (512 columns): tile t owns columns [256t, 256t + 128) for S / P and
 // [256t + 128, 256t + 256) for O.
+// The QK8 instantiation (H3_QK_E4M3) reads Q and K as e4m3 codes with one
+// static scale each and takes S with kind::f8f6f4 MMAs (half the tensor time
+// of the bf16 S, which sits on each tile's critical chain); P V stays bf16.
 #include "h3_internal.cuh"
 #include "ptx.cuh"
 
