@@ -91,6 +91,17 @@ def test_validation_rejects_bad_arguments_without_launch(lib):
     z = ctypes.c_void_p(16)
     assert lib.h3_attention(ctypes.byref(d), ctypes.byref(r), z, z, z, None, None, None, 0, z, None) == \
         h3.H3_ERR_UNSUPPORTED
+    # e4m3 q, k: attention needs the norm weights (their scales), unknown
+    # flags are refused, and the bf16 QKV call cannot write e4m3 codes
+    qk8 = h3.H3_QK_NORM_ROPE_IN_QKV | h3.H3_QK_E4M3
+    assert lib.h3_attention(ctypes.byref(d), ctypes.byref(r), z, z, z, None, None, None, qk8, z, None) == \
+        h3.H3_ERR_NULL
+    assert lib.h3_attention(ctypes.byref(d), ctypes.byref(r), z, z, z, z, z, None, h3.H3_QK_NORM_ROPE_IN_QKV | 8, z,
+                            None) == h3.H3_ERR_UNSUPPORTED
+    assert lib.h3_qkv_qknorm_mrope(ctypes.byref(d), ctypes.byref(r), z, z, z, z, z, qk8, z, z, z, None) == \
+        h3.H3_ERR_UNSUPPORTED
+    assert lib.h3_qkv_qknorm_mrope_e4m3(ctypes.byref(d), ctypes.byref(r), z, z, z, z, z, z, z,
+                                        h3.H3_QK_NORM_ROPE_IN_QKV | 8, z, z, z, None) == h3.H3_ERR_UNSUPPORTED
     # embed: video count must match the latent grid
     rc = lib.h3_embed_pack(ctypes.byref(d), ctypes.byref(r), z, 256, z, 2, 8, 6, 24, z, 2, 8, 64, z, z, z, z, z, z,
                            z, None)
