@@ -11,6 +11,12 @@ weak scaling, value = tokens of all ranks / max-over-ranks time.
 
 --impl reference times the float64 CPU oracle on a bounded sample of the same
 workload (the reference arm of this comparison; it is not tuned).
+
+Separate lines (one GPU each, not the headline): --e4m3 (the block's four
+GEMMs on e4m3 operands; with --qk-e4m3 also attention's Q K^T on e4m3
+codes), --sampler (the 50-block, 8-step layered sampler on 768x1344_5s;
+combinable with --e4m3 [--qk-e4m3]), --only CALL (one C-ABI call alone, for
+ncu captures; prints a timing line, not the JSON contract line).
 """
 from __future__ import annotations
 
