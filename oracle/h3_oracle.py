@@ -30,9 +30,11 @@ Readings adopted where the pages are silent or garbled:
   G12 x0 = x - sigma v, Euler x += (sigma' - sigma) v; G13 uniform sigmas with
   shift s*sigma / (1 + (s-1) sigma).
 
-Parity pins: every function here is pinned by tests/test_oracle_*.py except
-`head_unpack`, whose form is a reading (G11): parity unpinned beyond its shapes
-and the unpatchify round trip.
+Parity pins: every function here is pinned by tests/test_oracle_*.py.
+`head_unpack` computes what reading G11 states and is pinned to that
+statement composed from library routines; the reading itself (a non-affine LN
+and one linear per modality, no final modulation) has nothing on the pages to
+pin it against.
 """
 from __future__ import annotations
 
@@ -357,7 +359,7 @@ def block_forward_rows(x, mod, ranges, pos, rows, Wqkv, qn_w, kn_w, Wo, Wgu, Wd,
 
 
 # --------------------------------------------------------------------------
-# A10  output head (reading G11: parity unpinned beyond shapes)
+# A10  output head (reading G11; pinned to the reading's library composition)
 # --------------------------------------------------------------------------
 
 def head_unpack(x, ranges, W_vhead, W_ahead, t_lat, h_lat, w_lat, audio_channels, n_audio):

@@ -417,8 +417,57 @@ def test_euler_and_clean_latent_follow_rf_path():
         _pin_close(x, eps - v, 1e-13)
 
 
+def test_embed_matches_library_composition():
+    """The residual stream the embed assembles, rebuilt from library routines:
+    each modality's features through torch's linear, the audio latents made
+    channel-major by an einops rearrange ((channel, latent) -> token, G6), the
+    video by the 1x2x2 patchify rearrange, and the three blocks concatenated
+    text -> audio -> video (G1).  Odd, unequal sizes everywhere so that a
+    swapped range, an interleaved audio reshape or a transposed weight fails."""
+    import einops
+    rng = np.random.default_rng(21)
+    n_text, d_text, ch, n_aud, c_aud, T, Hl, Wl, D = 5, 7, 2, 3, 11, 2, 4, 6, 9
+    text = rng.standard_normal((n_text, d_text))
+    audio = rng.standard_normal((ch, n_aud, c_aud))
+    video = rng.standard_normal((T, Hl, Wl, 24))
+    W_text, W_aud, W_vid = (rng.standard_normal((D, k)) for k in (d_text, c_aud, 96))
+    r = O.pack_ranges(n_text, ch * n_aud, T * (Hl // 2) * (Wl // 2))
+    t = torch.from_numpy
+    ref = torch.cat([TF.linear(t(text), t(W_text)),
+                     TF.linear(t(einops.rearrange(audio, "c n d -> (c n) d")), t(W_aud)),
+                     TF.linear(t(einops.rearrange(video, "t (i ph) (j pw) c -> (t i j) (ph pw c)", ph=2, pw=2)),
+                               t(W_vid))])
+    _pin_close(O.embed(text, video, audio, W_text, W_vid, W_aud, r), ref.numpy(), 1e-12)
+    # modality ids: the same three blocks as a run-length expansion
+    ids = torch.repeat_interleave(torch.tensor([O.TEXT, O.AUDIO, O.VIDEO]), torch.tensor(r["count"]))
+    assert np.array_equal(O.modality_of_rows(r), ids.numpy())
+
+
+def test_head_unpack_matches_library_composition():
+    """The head rebuilt from library routines: torch's non-affine layer_norm
+    (eps 1e-6), the packed rows split by modality counts, torch's linear per
+    modality, and the inverse rearranges of the patchify and of the
+    channel-major audio packing.  Non-square head weights and unequal sizes, so
+    a transposed weight or a wrong reshape fails."""
+    import einops
+    rng = np.random.default_rng(22)
+    ch, n_aud, c_aud, T, Hl, Wl, D = 2, 5, 13, 2, 4, 6, 40
+    r = O.pack_ranges(3, ch * n_aud, T * (Hl // 2) * (Wl // 2))
+    x = rng.standard_normal((r["L"], D)) * 3 + 1
+    Wv, Wa = rng.standard_normal((96, D)), rng.standard_normal((c_aud, D))
+    vv, va = O.head_unpack(x, r, Wv, Wa, T, Hl, Wl, ch, n_aud)
+    t = torch.from_numpy
+    h = TF.layer_norm(t(x), (D,), eps=1e-6)
+    _, ha, hv = torch.split(h, r["count"])
+    ref_v = einops.rearrange(TF.linear(hv, t(Wv)).numpy(), "(t i j) (ph pw c) -> t (i ph) (j pw) c",
+                             t=T, i=Hl // 2, j=Wl // 2, ph=2, pw=2)
+    ref_a = einops.rearrange(TF.linear(ha, t(Wa)).numpy(), "(c n) d -> c n d", c=ch)
+    _pin_close(vv, ref_v, 1e-11)
+    _pin_close(va, ref_a, 1e-11)
+
+
 def test_head_unpack_shapes_and_roundtrip():
-    """Head form is a reading (parity unpinned beyond shapes and gather)."""
+    """Head shapes and the gather round trip (its form is a reading, G11)."""
     rng = np.random.default_rng(16)
     r = O.pack_ranges(3, 2 * 5, 2 * 2 * 3)
     D = 16
