@@ -203,9 +203,11 @@ __device__ __forceinline__ void qk_e4m3_inv_scales(const GemmEpilogue& e, float*
     mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
     mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
   }
+  // an all-zero norm weight makes every q (k) element 0: inverse scale 0
+  // (codes 0, no 0 * inf), and attention's scale product is 0 as well
   if (lane == 0) {
-    qk_inv[0] = 448.0f / (11.3137085f * mq);
-    qk_inv[1] = 448.0f / (11.3137085f * mk);
+    qk_inv[0] = mq > 0.f ? 448.0f / (11.3137085f * mq) : 0.f;
+    qk_inv[1] = mk > 0.f ? 448.0f / (11.3137085f * mk) : 0.f;
   }
 }
 

@@ -153,6 +153,10 @@ def qk_code_scale(w) -> tuple[np.float32, np.float32]:
     """(inverse scale, scale) of the e4m3 codes of q or k rows normalised
     with weight w (see the module docstring), in fp32."""
     m = np.float32(np.max(np.abs(np.asarray(w, np.float32))))
+    if m == 0:
+        # an all-zero weight makes every element 0: codes 0 and scale 0
+        # (the scaling of F2 for a zero row)
+        return np.float32(0.0), np.float32(0.0)
     d = np.float32(QK_SQRT128 * m)
     return np.float32(np.float32(448.0) / d), np.float32(d / np.float32(448.0))
 

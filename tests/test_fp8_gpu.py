@@ -287,6 +287,41 @@ def test_attention_e4m3_qk(L):
     assert np.all(got[L:] == 0)
 
 
+def test_e4m3_qk_zero_norm_weight():
+    """An all-zero q norm weight: every q element is 0, so its e4m3 codes are
+    0 (inverse scale 0, not 0 * inf) and attention is the plain average of v
+    over the valid keys, as the bf16 path gives; nothing turns NaN."""
+    w = S.WORKLOADS["tiny"]
+    inp = _inputs(w)
+    Wq, Ws = _weights_e4m3(w)["Wqkv"]
+    r, pos = oracle_ranges_and_pos(w)
+    L, Lp = r["L"], r["L_pad"]
+    rng = np.random.default_rng(505)
+    xq, xs = F8.quantize_rows(_rows(rng, L, Lp, w.D))
+    d, rg = _dims(w, r)
+    zero_w = np.zeros(128, np.float32)
+    assert F8.qk_code_scale(zero_w) == (0.0, 0.0)
+    q8, k8 = (torch.full((w.H, Lp, 128), 0x55, dtype=torch.uint8, device=DEV) for _ in range(2))
+    v = torch.empty(w.H, Lp, 128, dtype=torch.bfloat16, device=DEV)
+    pos_pad = np.zeros((Lp, 3), np.float32)
+    pos_pad[:L] = pos
+    zw = to_dev_bf16(zero_w, DEV)
+    kn = to_dev_bf16(inp["kn_w"], DEV)
+    flags = h3.H3_QK_NORM_ROPE_IN_QKV | h3.H3_QK_E4M3
+    h3.h3_qkv_qknorm_mrope_e4m3(d, rg, _u8(xq), _f32(xs), _u8(Wq), _f32(Ws), zw, kn, _f32(pos_pad), q8, k8, v,
+                                flags=flags)
+    o = torch.empty(Lp, w.H * 128, dtype=torch.bfloat16, device=DEV)
+    h3.h3_attention(d, rg, q8, k8, v, o, qn_w=zw, kn_w=kn, flags=flags)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    assert np.all(F8.e4m3_decode(to_np(q8)) == 0)
+    got = to_np(o)
+    assert np.all(np.isfinite(got))
+    vv = to_np(v)[:, :L, :]                                   # [H, L, 128]
+    ref = np.broadcast_to(vv.mean(axis=1)[None], (L, w.H, 128)).reshape(L, w.H * 128)
+    check_close(got[:L], ref, "attention with a zero q norm weight")
+
+
 @pytest.mark.parametrize("qk_e4m3", [False, True], ids=["qk_bf16", "qk_e4m3"])
 @pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
 def test_block_e4m3_against_oracle(w, qk_e4m3):

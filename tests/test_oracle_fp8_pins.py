@@ -146,3 +146,16 @@ def test_qk_codes_static_scale():
     codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
     vals = F.e4m3_decode(codes) * np.float64(s)
     assert np.array_equal(F.quantize_qk(vals, w) & 0x7F, codes & 0x7F)
+
+
+def test_qk_codes_zero_norm_weight():
+    """An all-zero norm weight (every q or k element 0) takes the zero-row
+    rule of the row scaling: inverse scale 0 and scale 0, so its codes are 0
+    and dequantise to 0, with no 0 * inf anywhere."""
+    inv, s = F.qk_code_scale(np.zeros(128, np.float32))
+    assert inv == 0.0 and s == 0.0
+    x = np.zeros((3, 128))
+    x[1, 7] = -0.0
+    c = F.quantize_qk(x, np.zeros(128, np.float32))
+    assert np.all((c & 0x7F) == 0)
+    assert np.all(F.dequantize_qk(c, np.zeros(128, np.float32)) == 0)
