@@ -95,6 +95,62 @@ def test_sampler_e4m3_against_oracle(qk_e4m3):
     check_close(ga, ra, "audio latent")
 
 
+def test_full_width_two_block_stack_one_step_sampled_rows():
+    """Two full-width blocks and one Euler step (sigma 1 -> 0) on the 768sq_2s
+    workload (7,904 packed tokens), through the sampler's calls.  The oracle
+    runs the first block on every row (the second block's attention reads all
+    of its output), then the second block, the head and the Euler update on
+    sampled rows; the test compares the latent entries that those rows
+    produce (a video token's 2 x 2 x 24 latent values, an audio token's 64)."""
+    w, n_layers, n_steps = S.WORKLOADS["768sq_2s"], 2, 1
+    inp = S.make_inputs(w)
+    st = S.make_stack_inputs(w, n_layers, n_steps)
+    dev = torch.device("cuda", 0)
+    blocks = [{k: to_dev_bf16(v, dev) for k, v in b.items()} for b in st["blocks"]]
+    smp = H3Sampler(w, inp, blocks, device=dev)
+    text = to_dev_bf16(inp["text"], dev)
+    lv = torch.from_numpy(st["lat_video"]).to(dev)
+    la = torch.from_numpy(st["lat_audio"]).to(dev)
+    lv_bf, la_bf = lv.to(torch.bfloat16), la.to(torch.bfloat16)
+    mod_all = torch.from_numpy(st["mod_all"]).to(dev)
+    smp.run(text, lv, la, lv_bf, la_bf, mod_all, n_steps)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    del blocks, smp
+    r, pos = oracle_ranges_and_pos(w)
+    L = r["L"]
+    T, Hl, Wl, _ = st["lat_video"].shape
+    ch, na, _ = st["lat_audio"].shape
+    x = O.embed(inp["text"], O.round_to_bf16(st["lat_video"]), O.round_to_bf16(st["lat_audio"]), inp["W_text"],
+                inp["W_vid"], inp["W_aud"], r)
+    b0, b1 = st["blocks"]
+    x = O.block_forward(x, st["mod_all"][0][0], r, pos, n_heads=w.H, **b0)
+    sa_, ca_ = r["start"][O.AUDIO], r["count"][O.AUDIO]
+    sv_, cv_ = r["start"][O.VIDEO], r["count"][O.VIDEO]
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([rng.choice(np.arange(sa_, sa_ + ca_), 6, replace=False),
+                                     rng.choice(np.arange(sv_, sv_ + cv_), 18, replace=False),
+                                     [sa_, sa_ + ca_ - 1, sv_, L - 1]]))
+    x2, _ = O.block_forward_rows(x, st["mod_all"][0][1], r, pos, rows, n_heads=w.H, **b1)
+    # the head is row-local: run it on a stream that holds only the sampled
+    # rows, then keep the latent entries those rows produce
+    xs = np.zeros((L, w.D))
+    xs[rows] = x2
+    vv, va = O.head_unpack(xs, r, inp["W_vhead"], inp["W_ahead"], T, Hl, Wl, ch, na)
+    rv = O.euler_step(st["lat_video"], vv, 1.0, 0.0)
+    ra = O.euler_step(st["lat_audio"], va, 1.0, 0.0)
+    src = np.zeros(L, bool)
+    src[rows] = True
+    sel_v = O.unpatchify(np.repeat(src[sv_:sv_ + cv_, None], 96, axis=1), T, Hl, Wl)
+    sel_a = src[sa_:sa_ + ca_].reshape(ch, na)
+    assert sel_v.sum() > 0 and sel_a.sum() > 0
+    gv, ga = to_np(lv), to_np(la)
+    for name, g, ref, lat0 in (("video", gv[sel_v], rv[sel_v], st["lat_video"][sel_v]),
+                               ("audio", ga[sel_a], ra[sel_a], st["lat_audio"][sel_a])):
+        check_close(g - lat0, ref - lat0, f"{name} latent change (sampled tokens)")
+        check_close(g, ref, f"{name} latent (sampled tokens)")
+
+
 def test_sampler_checkpoint_resume_is_bit_exact(tmp_path):
     """Stopping after two of four steps, saving the state, loading it into
     fresh tensors and resuming gives the uninterrupted run's latents bit for
