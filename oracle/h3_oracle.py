@@ -28,7 +28,8 @@ Readings adopted where the pages are silent or garbled:
   [modality][shift_msa, scale_msa, gate_msa, shift_mlp, scale_mlp, gate_mlp][D];
   G10 no biases; G11 head = non-affine LN + per-modality linear;
   G12 x0 = x - sigma v, Euler x += (sigma' - sigma) v; G13 uniform sigmas with
-  shift s*sigma / (1 + (s-1) sigma).
+  shift s*sigma / (1 + (s-1) sigma); G22 AdaLN producer = SiLU then one
+  linear per block from a D/2-wide conditioning vector to 18 D.
 
 Parity pins: every function here is pinned by tests/test_oracle_*.py.
 `head_unpack` computes what reading G11 states and is pinned to that
@@ -371,6 +372,21 @@ def head_unpack(x, ranges, W_vhead, W_ahead, t_lat, h_lat, w_lat, audio_channels
     v_video = unpatchify(linear(h[sv:sv + cv], W_vhead), t_lat, h_lat, w_lat)
     v_audio = linear(h[sa:sa + ca], W_ahead).reshape(audio_channels, n_audio, np.asarray(W_ahead).shape[0])
     return v_video, v_audio
+
+
+# --------------------------------------------------------------------------
+# NEXT-3  AdaLN modulation producer (reading G22)
+# --------------------------------------------------------------------------
+
+def adaln_modulation(c, W, D: int) -> np.ndarray:
+    """The modulation of one block from conditioning vectors c [n, C]
+    (timestep + condition embedding; the pages say the AdaLN outputs depend
+    on these alone and can be precomputed [gojay §5; shouss §3.1]): SiLU, then
+    the block's own linear W [18 D, C] (no bias, G10), read as
+    [3 modalities][shift_msa, scale_msa, gate_msa, shift_mlp, scale_mlp,
+    gate_mlp][D] (G9).  Returns [n, 3, 6, D]."""
+    c = np.atleast_2d(np.asarray(c, np.float64))
+    return linear(silu(c), W).reshape(c.shape[0], 3, 6, D)
 
 
 # --------------------------------------------------------------------------

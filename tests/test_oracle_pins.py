@@ -41,6 +41,42 @@ def test_config_widths_from_pages(golden):
         int(golden["ffn_inner"]), int(golden["text_input_dim"]))
 
 
+def test_adaln_producer_width_matches_page_parameter_counts(golden):
+    """Reading G22: each block's AdaLN producer is one linear from a D/2-wide
+    conditioning vector to the 18 D modulation features.  That width is the
+    one that reproduces the pages' counts: 50 blocks x 18 D x D/2 = 13.0 B
+    parameters in the AdaLN branch, and with the blocks' attention and FFN
+    weights (19.3 B) the 33 B total and the ~20 B deployed without it."""
+    D, blocks = int(golden["hidden"]), int(golden["blocks"])
+    I, F = int(golden["attention_inner"]), int(golden["ffn_inner"])
+    adaln = blocks * 18 * D * (D // 2)
+    trunk = blocks * (D * 3 * I + I * D + 2 * D * F + F * D)
+    assert abs(adaln / 1e9 - float(golden["adaln_params_billion"])) < 0.01 * 13
+    assert abs(trunk / 1e9 - float(golden["deploy_params_billion"])) < 0.05 * 20
+    assert abs((adaln + trunk) / 1e9 - float(golden["transformer_params_billion"])) < 0.05 * 33
+
+
+def test_adaln_producer_matches_library_composition():
+    """SiLU then linear, read as [n][3][6][D], against torch's silu and
+    linear; and each (modality, slot) block of W's rows drives exactly that
+    slice of the modulation."""
+    rng = np.random.default_rng(23)
+    D, C, n = 8, 5, 3
+    c = rng.standard_normal((n, C)) * 2
+    W = rng.standard_normal((18 * D, C))
+    got = O.adaln_modulation(c, W, D)
+    ref = TF.linear(TF.silu(torch.from_numpy(c)), torch.from_numpy(W)).reshape(n, 3, 6, D)
+    _pin_close(got, ref.numpy(), 1e-12)
+    for m in range(3):
+        for j in range(6):
+            W1 = np.zeros_like(W)
+            W1[(m * 6 + j) * D:(m * 6 + j + 1) * D] = W[(m * 6 + j) * D:(m * 6 + j + 1) * D]
+            g1 = O.adaln_modulation(c, W1, D)
+            mask = np.zeros((3, 6), bool)
+            mask[m, j] = True
+            assert np.all(g1[:, ~mask] == 0) and np.all(g1[:, mask] != 0)
+
+
 def test_modulation_uses_each_of_18D_slices_once():
     """Perturbing any one of the 3x6 slices of mod changes exactly the output
     that slice should drive, and only for that modality's rows."""
