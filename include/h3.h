@@ -210,17 +210,51 @@ int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x,
                    const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
                    int C_audio, h3_bf16* hn, float* v_video, float* v_audio, void* stream);
 
+/* A10 + A11 fused: the head of h3_head_unpack with the Euler step of each
+ * latent in its GEMM epilogues, so the velocities are never written out:
+ *   lat_video += (sigma_video_next - sigma_video) * v_video,
+ *   lat_audio += (sigma_audio_next - sigma_audio) * v_audio,
+ * with v_video, v_audio as h3_head_unpack computes them (same accumulation;
+ * the update is the same fused multiply-add as h3_euler_step, so the result
+ * equals h3_head_unpack followed by h3_euler_step on each latent bit for
+ * bit).  Each modality has its own sigmas (its own shifted schedule,
+ * [shouss] §6); text rows are not touched ([shouss] §5).  lat_video
+ * [T][Hl][Wl][C_lat] and lat_audio [audio_channels][n_audio][C_audio] are
+ * fp32 device arrays updated in place; lat_video_bf16 / lat_audio_bf16, when
+ * not NULL, receive the updated latents rounded to bf16 (the next step's
+ * transformer input), same layouts.  hn [L_pad][D] bf16 scratch.  Errors as
+ * h3_head_unpack. */
+int h3_head_euler(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
+                  const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
+                  int C_audio, h3_bf16* hn, float* lat_video, float* lat_audio, float sigma_video,
+                  float sigma_video_next, float sigma_audio, float sigma_audio_next, h3_bf16* lat_video_bf16,
+                  h3_bf16* lat_audio_bf16, void* stream);
+
+/* NEXT-3 (a reading, G22): the AdaLN modulation producer of one block.
+ * The pages put ~13B parameters in the AdaLN branch and say its outputs
+ * depend only on the timestep and the condition, so they can be computed
+ * ahead and cached ([gojay] §5; [shouss] §3.1: 6D features per modality,
+ * 18D in all).  Read here as one linear per block on SiLU of a conditioning
+ * vector (timestep + condition embedding, computed by the caller; its width
+ * D/2 reproduces the 13B count at 50 blocks), no bias:
+ *   mod[i] = W * SiLU(c[i]), viewed as [3][6][D] (layout of mod elsewhere).
+ *   c   [n][c_dim] fp32 device (n >= 1 vectors, e.g. one per sampler step)
+ *   W   [18 D][c_dim] bf16 device, c_dim a multiple of 8
+ *   ws  scratch of h3_adaln_workspace_bytes(n, c_dim) bytes (SiLU(c) in bf16)
+ *   mod [n][3][6][D] fp32 device output, rows ld_mod floats apart (0: 18 D;
+ *       e.g. n_blocks * 18 D to fill block b's column of a
+ *       [step][block][3][6][D] cache, mod pointing at block b)
+ * SiLU(c) enters the tensor-core GEMM as bf16 (fp32 accumulation).
+ * Errors: H3_ERR_SHAPE (n <= 0), H3_ERR_UNSUPPORTED (c_dim), NULL / alignment
+ * as elsewhere; nothing is launched on error. */
+size_t h3_adaln_workspace_bytes(int n, int c_dim);
+int h3_adaln_modulation(const h3_dims* dims, const float* c, int n, int c_dim, const h3_bf16* W, h3_bf16* ws,
+                        float* mod, int64_t ld_mod, void* stream);
+
 /* A11.  lat[i] += (sigma_next - sigma) * vel[i] for i < n: one Euler step of
  * the rectified-flow ODE on a generation target (x0 = x - sigma v;
  * [shouss] §5, §6).  lat, vel: fp32 device arrays of n elements. */
 int h3_euler_step(float* lat, const float* vel, int64_t n, float sigma, float sigma_next, void* stream);
-
-/* Diagnostic: y[i] = 2^x[i] on the FMA pipe instead of the MUFU unit (the
- * form measured for part of attention's softmax exponentials, which took
- * longer there): x clamped to >= -125, x = j + f with j = rint(x), 2^f from a
- * cubic (max relative error 7.5e-5 for x in [-125, 64]), 2^j added to the
- * exponent.  x, y: fp32 device arrays of n elements. */
-int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream);
 
 /* Block weights and scratch buffers for h3_block_forward (all device
  * pointers, layouts as in the individual calls). */

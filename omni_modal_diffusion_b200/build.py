@@ -57,6 +57,28 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     return LIB
 
 
+PROBE_SRC = os.path.join(ROOT, "tests", "cuda", "exp2_fma2_probe.cu")
+PROBE_LIB = os.path.join(ROOT, "tests", "cuda", "libexp2_probe.so")
+
+
+def build_probe(force: bool = False) -> str:
+    """The test-only probe library (tests/cuda): the attention softmax's
+    FMA-pipe exponential over an array, for its error-bound test.  Not part of
+    libh3.so."""
+    deps = [PROBE_SRC, os.path.join(PKG, "csrc", "ptx.cuh")]
+    if not force and os.path.exists(PROBE_LIB) and all(os.path.getmtime(s) <= os.path.getmtime(PROBE_LIB)
+                                                         for s in deps):
+        return PROBE_LIB
+    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-shared",
+           "-o", PROBE_LIB + ".tmp", PROBE_SRC]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
+    os.replace(PROBE_LIB + ".tmp", PROBE_LIB)
+    return PROBE_LIB
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
+    build_probe(force="--force" in sys.argv)
     print(LIB)

@@ -19,6 +19,15 @@
 //              back over S in TMEM as packed bf16 in two halves of 64 keys,
 //              each released to the PV MMA as soon as it is stored, finally
 //              O / l to global memory.
+// The two softmax warpgroups take turns: tile 1's exponentials of key tile j
+// start when tile 0's have finished, tile 0's of key tile j + 1 when tile 1's
+// of j have (an mbarrier handoff), so each phase has the MUFU units and the
+// issue slots of all four sub-partitions to itself while the tensor core runs
+// the other tile's P V and next S.  A fixed share of each row's exponentials
+// (H3_ATTN_POLY_COLS of every 16 columns) is taken on the FMA pipe instead
+// (exp2_fma2), which shortens a phase below the MUFU-only 1,024 clocks of a
+// 128 x 128 tile (16 exponentials per clock per SM).
+// With an odd number of query tiles the last CTA runs tile 0 alone.
 // TMEM (512 columns): tile t owns columns [256t, 256t + 128) for S / P and
 // [256t + 128, 256t + 256) for O.
 // The QK8 instantiation (H3_QK_E4M3) reads Q and K as e4m3 codes with one
@@ -46,17 +55,43 @@ constexpr int NUM_THREADS = 320;
 constexpr int TILE = 128;
 constexpr int HALF_BYTES = TILE * 64 * 2;   // 128 rows x 64 bf16 = 16 KB
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 32 KB
+// Stages of the V ring (2 or 3).  K keeps 2: a K tile is needed one key step
+// later than the V tile loaded before it.
+#ifndef H3_ATTN_V_STAGES
+#define H3_ATTN_V_STAGES 2
+#endif
+constexpr int VS = H3_ATTN_V_STAGES;
+static_assert(VS == 2 || VS == 3, "H3_ATTN_V_STAGES: 2 or 3");
 // Q and K tiles: bf16 (32 KB, two 64-column halves) or, with QK8, e4m3 codes
 // (16 KB, one 128-byte row per token)
 template <bool QK8> struct Layout {
   static constexpr int QK_TILE = QK8 ? TILE * 128 : TILE_BYTES;
   static constexpr int Q = 0;                  // 2 query tiles
   static constexpr int K = Q + 2 * QK_TILE;    // 2 stages
-  static constexpr int V = K + 2 * QK_TILE;    // 2 stages
-  static constexpr int BAR = V + 2 * TILE_BYTES;
+  static constexpr int V = K + 2 * QK_TILE;    // VS stages
+  static constexpr int BAR = V + VS * TILE_BYTES;
   static constexpr int BYTES = BAR + 256 + 1024;
+  static_assert(BYTES <= 232448, "shared memory per CTA");
 };
 constexpr int TMEM_COLS = 512;
+// Of every 16 key columns of a row, how many take their exponential on the
+// FMA pipe (exp2_fma2) instead of the MUFU unit (0..16, even).
+#ifndef H3_ATTN_POLY_COLS
+#define H3_ATTN_POLY_COLS 0
+#endif
+static_assert(H3_ATTN_POLY_COLS >= 0 && H3_ATTN_POLY_COLS <= 16 && H3_ATTN_POLY_COLS % 2 == 0,
+              "H3_ATTN_POLY_COLS: an even count of 0..16");
+// The two softmax warpgroups take turns on the exponentials (1) or run
+// whenever their S is ready (0).
+#ifndef H3_ATTN_TURNS
+#define H3_ATTN_TURNS 0
+#endif
+// S is read from TMEM in two 64-key halves (1: half 1 is loaded while P of
+// half 0 is stored, and only 64 scores are live in registers at a time) or
+// whole (0).
+#ifndef H3_ATTN_S_HALVES
+#define H3_ATTN_S_HALVES 1
+#endif
 // A 64-key half whose exponentials (against the current reference) sum past
 // this moves the reference: every p of an accepted half is <= 2^16, so p, the
 // row sum and O stay far from the fp32 range (and bf16 P keeps its relative
@@ -103,21 +138,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2] per K stage
-  uint64_t* v_full = bars + 3;    // [2] per V stage
-  uint64_t* k_empty = bars + 5;   // [2] per K stage: freed after the tile's last S MMA
-  uint64_t* v_empty = bars + 7;   // [2] per V stage: freed after the tile's last PV MMA
-  uint64_t* s_full = bars + 9;    // [2] per query tile
-  uint64_t* o_final = bars + 11;  // [2] per query tile
-  uint64_t* p_full = bars + 13;   // [2 tiles][2 halves of the key tile]: P half in TMEM (4 warp arrivals)
-  uint64_t* drain = bars + 17;    // the MMA issuer's last commit before teardown
-  uint64_t* pv0_done = bars + 18; // [2] per query tile: PV on the first key half complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
-  float* qk_scale = reinterpret_cast<float*>(bars + 21);  // QK8: dequantisation of S
+  uint64_t* k_empty = bars + 3;   // [2] per K stage: freed after the tile's last S MMA
+  uint64_t* v_full = bars + 5;    // [VS] per V stage
+  uint64_t* v_empty = bars + 8;   // [VS] per V stage: freed after the tile's last PV MMA
+  uint64_t* s_full = bars + 11;   // [2] per query tile
+  uint64_t* o_final = bars + 13;  // [2] per query tile
+  uint64_t* p_full = bars + 15;   // [2 tiles][2 halves of the key tile]: P half in TMEM (4 warp arrivals)
+  uint64_t* drain = bars + 19;    // the MMA issuer's last commit before teardown
+  uint64_t* pv0_done = bars + 20; // [2] per query tile: PV on the first key half complete
+  uint64_t* turn = bars + 22;     // [2] per query tile: its exponentials of a key tile done (4 warp arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  float* qk_scale = reinterpret_cast<float*>(bars + 25);  // QK8: dequantisation of S
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
   const int qt0 = blockIdx.x * 2;
-  const int qt1 = (qt0 + 1 < n_qt) ? qt0 + 1 : qt0;  // odd tile count: tile 1 recomputes tile 0, not stored
+  const bool two = qt0 + 1 < n_qt;  // odd tile count: the last CTA has tile 0 only
+  const int nt = two ? 2 : 1;
+  const int qt1 = two ? qt0 + 1 : qt0;
   const int h = blockIdx.y;
   const int nkv = (L + TILE - 1) / TILE;
   const int row0 = h * L_pad;
@@ -126,14 +164,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
       mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[2 * s], 4);
       mbar_init(&p_full[2 * s + 1], 4);
       mbar_init(&pv0_done[s], 1);
       mbar_init(&o_final[s], 1);
+      mbar_init(&turn[s], 4);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -167,36 +208,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * QK_TILE);
-      if (QK8) {
-        tma_load_2d(sQ, &tmQ, q_full, 0, row0 + qt0 * TILE);
-        tma_load_2d(sQ + QK_TILE, &tmQ, q_full, 0, row0 + qt1 * TILE);
-      } else {
-        tma_load_2d(sQ, &tmQ, q_full, 0, row0 + qt0 * TILE);
-        tma_load_2d(sQ + HALF_BYTES, &tmQ, q_full, 64, row0 + qt0 * TILE);
-        tma_load_2d(sQ + TILE_BYTES, &tmQ, q_full, 0, row0 + qt1 * TILE);
-        tma_load_2d(sQ + TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, row0 + qt1 * TILE);
+      mbar_arrive_expect_tx(q_full, nt * QK_TILE);
+      for (int t = 0; t < nt; ++t) {
+        const int qrow = row0 + (t == 0 ? qt0 : qt1) * TILE;
+        tma_load_2d(sQ + t * QK_TILE, &tmQ, q_full, 0, qrow);
+        if (!QK8) tma_load_2d(sQ + t * QK_TILE + HALF_BYTES, &tmQ, q_full, 64, qrow);
       }
       long long k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
         uint8_t* dk = sK + st * QK_TILE;
-        uint8_t* dv = sV + st * TILE_BYTES;
+        const int sv = j % VS;
+        uint8_t* dv = sV + sv * TILE_BYTES;
         if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&k_full[st], QK_TILE);
         tma_load_2d(dk, &tmK, &k_full[st], 0, row0 + j * TILE);
         if (!QK8) tma_load_2d(dk + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
         ++k_issued;
-        if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1)) break;
-        mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
-        tma_load_2d(dv, &tmV, &v_full[st], 0, row0 + j * TILE);
-        tma_load_2d(dv + HALF_BYTES, &tmV, &v_full[st], 64, row0 + j * TILE);
+        if (!mbar_wait(&v_empty[sv], ((j / VS) & 1) ^ 1)) break;
+        mbar_arrive_expect_tx(&v_full[sv], TILE_BYTES);
+        tma_load_2d(dv, &tmV, &v_full[sv], 0, row0 + j * TILE);
+        tma_load_2d(dv + HALF_BYTES, &tmV, &v_full[sv], 64, row0 + j * TILE);
         ++v_issued;
       }
       // every load of this CTA has landed before it leaves
       mbar_wait(q_full, 0);
       drain_loads(k_full, 2, k_issued);
-      drain_loads(v_full, 2, v_issued);
+      drain_loads(v_full, VS, v_issued);
     }
   } else if (warp == 1) {
     // The whole warp runs the issue loop, converged; one elected lane issues.
@@ -230,7 +268,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // O_t += P_t V_j for keys [64 hf, 64 hf + 64): P_t (bf16, two per column)
     // read from TMEM columns [32 hf, 32 hf + 32) where S_t was
     auto issue_pv_half = [&](int t, int j, int hf) {
-      const uint64_t vd = v_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
+      const uint64_t vd = v_desc + (uint64_t)(((j % VS) * TILE_BYTES) >> 4);
 #pragma unroll
       for (int k4 = 0; k4 < 4; ++k4) {
         const int kk = hf * 4 + k4;
@@ -242,17 +280,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok) {
       tc_fence_after();
       issue_s(0, 0);
-      issue_s(1, 0);
+      if (two) issue_s(1, 0);
       umma_commit(&k_empty[0]);
     }
     for (int j = 0; j < nkv && ok; ++j) {
       const bool more = j + 1 < nkv;
-      for (int t = 0; t < 2 && ok; ++t) {
+      for (int t = 0; t < nt && ok; ++t) {
         // P is released in two halves: PV on keys [0, 64) runs while the
         // softmax warps still take the second half's exponentials
         for (int hf = 0; hf < 2; ++hf) {
           if (!MMA_WAIT_WARP(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
-          if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j & 1], (j >> 1) & 1)) { ok = false; break; }
+          if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j % VS], (j / VS) & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv_half(t, j, hf);
           if (hf == 0) umma_commit(&pv0_done[t]);
@@ -264,18 +302,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
           }
           issue_s(t, j + 1);
-          if (t == 1) umma_commit(&k_empty[(j + 1) & 1]);
+          if (t == nt - 1) umma_commit(&k_empty[(j + 1) & 1]);
         } else {
           umma_commit(&o_final[t]);
         }
       }
-      umma_commit(&v_empty[j & 1]);
+      umma_commit(&v_empty[j % VS]);
     }
     drain_mmas(drain);
-  } else {
+  } else if ((warp - 2) >> 2 < nt) {
     const int t = (warp - 2) >> 2;  // query tile of this warpgroup
-    // log2(e) / sqrt(128), times the dequantisation of e4m3 S
-    const float sl2 = QK8 ? scale_log2 * *qk_scale : scale_log2;
+    // log2(e) / sqrt(128), times the dequantisation of e4m3 S.  A zero
+    // dequantisation (an all-zero norm weight: every code of q or k is 0,
+    // so S is 0) is raised to a tiny positive scale, so that masked keys
+    // (-inf) still give -inf and not 0 * inf = NaN: the softmax is uniform.
+    const float sl2 = QK8 ? fmaxf(scale_log2 * *qk_scale, 1e-30f) : scale_log2;
     const int qw = warp & 3;        // TMEM lane quarter this warp may access
     const int r = qw * 32 + lane;   // query row inside the tile
     const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
@@ -288,14 +329,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       float s[128];
+      constexpr int kFirstLoad = H3_ATTN_S_HALVES ? 2 : 4;  // 32-column chunks loaded up front
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
+      for (int c = 0; c < kFirstLoad; ++c) tmem_ld32(tS + c * 32, reinterpret_cast<uint32_t*>(s + c * 32));
       tmem_wait_ld();
 
       const int valid = L - j * TILE;  // keys [0, valid) of this tile are real
       if (valid < TILE) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 32 * kFirstLoad; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
       // row max over keys [c0, c0 + n)
@@ -317,20 +359,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // that half's row max, with O and the sums rescaled first.  A half that
       // passed the check lies within 2^16 of the reference, so it stays in
       // range when the reference moves up.  No per-tile row max otherwise.
-      if (j == 0) m_ref = row_max(0, 128) * sl2;
+      // (with S in halves: the first half's max; the second half of the
+      // first key tile then takes the overflow check like any later half)
+      if (j == 0) m_ref = row_max(0, 32 * kFirstLoad) * sl2;
+      // wait for the other tile's exponentials (of key tile j - 1 for tile 0,
+      // of key tile j for tile 1) to finish
+      if (H3_ATTN_TURNS && two && (t == 1 || j > 0)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&turn[1 - t], (uint32_t)((j - (t == 0 ? 1 : 0)) & 1)));
+        if (!ok) break;
+      }
       const uint64_t sc2 = f2_pack(sl2, sl2);
-      // p = 2^(s * sl2 - m_ref) on the MUFU unit (masked keys, -inf,
-      // give exactly 0); returns this row's sum over the half
-      auto exp_half = [&](int hf, uint32_t* pk) {
+      // p = 2^(s * sl2 - m_ref); returns this row's sum over the half.  The
+      // last key tile (masked keys at -inf, which give exactly 0) takes every
+      // exponential on the MUFU unit; the others take H3_ATTN_POLY_COLS of
+      // every 16 on the FMA pipe.
+      auto exp_half = [&](int hf, uint32_t* pk, auto poly_tag) {
+        constexpr bool kPoly = decltype(poly_tag)::value;
         const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+        const float pa = sl2 * (1.0f / 252.0f), pb = (125.0f - m_ref) * (1.0f / 252.0f);
         uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const int cc = hf * 64 + c;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[cc], s[cc + 1]), sc2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_pack(p0, p1));
+          uint64_t p2;
+          if (kPoly && (c & 15) < H3_ATTN_POLY_COLS) {
+            p2 = exp2_fma2(s[cc], s[cc + 1], pa, pb);
+          } else {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[cc], s[cc + 1]), sc2, nm2), x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], p2);
           pk[c / 2] = pack_bf16x2(p0, p1);
         }
         float a0, a1, a2, a3;
@@ -338,14 +399,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         f2_unpack(acc[1], a2, a3);
         return (a0 + a1) + (a2 + a3);
       };
+      auto exp_half_sel = [&](int hf, uint32_t* pk) {
+        if constexpr (H3_ATTN_POLY_COLS > 0)
+          return valid < TILE ? exp_half(hf, pk, std::false_type{}) : exp_half(hf, pk, std::true_type{});
+        else
+          return exp_half(hf, pk, std::false_type{});
+      };
       float hsum[2];
       // P for keys [64 hf, 64 hf + 64) goes to TMEM columns [32 hf, 32 hf + 32)
       // (it only overwrites S columns already in registers)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pk[32];
-        float hs = exp_half(hf, pk);
-        if (j > 0 && __any_sync(0xffffffffu, !(hs <= P_HALF_SUM_LIMIT))) {
+        if (H3_ATTN_S_HALVES && hf == 1) {
+          // the second half's scores, loaded while P of the first half was stored
+          tmem_wait_ld();
+          if (valid < TILE) {
+#pragma unroll
+            for (int c = 64; c < 128; ++c)
+              if (c >= valid) s[c] = -INFINITY;
+          }
+        }
+        float hs = exp_half_sel(hf, pk);
+        if ((j > 0 || (H3_ATTN_S_HALVES && hf == 1)) && __any_sync(0xffffffffu, !(hs <= P_HALF_SUM_LIMIT))) {
           // this half's scores again, from TMEM: P has not overwritten them
           // (P of keys [0, 64) goes to columns [0, 32))
           tmem_ld32(tS + hf * 64, reinterpret_cast<uint32_t*>(s + hf * 64));
@@ -378,9 +454,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tmem_wait_st();
           l_sum *= a;
-          hs = exp_half(hf, pk);
+          hs = exp_half_sel(hf, pk);
         }
         hsum[hf] = hs;
+        if (H3_ATTN_S_HALVES && hf == 0) {
+          // load the second half's scores (columns [64, 128), which no P
+          // store touches) while this half's P is stored
+          tmem_ld32(tS + 64, reinterpret_cast<uint32_t*>(s + 64));
+          tmem_ld32(tS + 96, reinterpret_cast<uint32_t*>(s + 96));
+        }
         tmem_st32(tS + hf * 32, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -388,11 +470,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[2 * t + hf]);
       }
       if (!ok) break;
+      if (H3_ATTN_TURNS && two && lane == 0) mbar_arrive(&turn[t]);
       l_sum += hsum[0] + hsum[1];
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
     const int qt = t == 0 ? qt0 : qt1;
-    if (ok && (t == 0 || qt1 != qt0)) {
+    if (ok) {
       tc_fence_after();
       const int grow = qt * TILE + r;
       const float inv = (grow < L) ? 1.0f / l_sum : 0.0f;

@@ -293,26 +293,25 @@ __global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
   mbar_wait_limit(&bar, 0, limit_ns);
 }
 
-// The attention softmax's FMA-pipe exponential on an array (for checking it
-// against its error bound).
-__global__ void exp2_fma_pipe_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
-  const long long pairs = n / 2;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < pairs;
-       i += (long long)gridDim.x * blockDim.x) {
-    float y0, y1;
-    exp2_poly2(x[2 * i], x[2 * i + 1], y0, y1);
-    y[2 * i] = y0;
-    y[2 * i + 1] = y1;
-  }
-  if (n & 1 && blockIdx.x == 0 && threadIdx.x == 0) {
-    float y0, y1;
-    exp2_poly2(x[n - 1], x[n - 1], y0, y1);
-    y[n - 1] = y0;
+// a[i] = bf16(SiLU(c[i])) = bf16(c / (1 + e^-c)): the conditioning vectors
+// of the AdaLN producer, as the A operand of its GEMM
+__global__ void silu_bf16_kernel(const float* __restrict__ c, long long n, bf16* __restrict__ a) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = c[i];
+    a[i] = __float2bfloat16_rn(v / (1.0f + expf(-v)));
   }
 }
 
 }  // namespace ew_detail
 using namespace ew_detail;
+
+cudaError_t launch_silu_bf16(const float* c, long long n, bf16* a, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148LL * 8) blocks = 148LL * 8;
+  silu_bf16_kernel<<<(int)blocks, 256, 0, stream>>>(c, n, a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const bf16* video, int T, int Hl, int Wl, int C_lat, int n_audio, int audio_channels,
                         const int* rstart, const int* rcount, int L, int L_pad, bf16* patches, float* pos,
@@ -374,15 +373,6 @@ cudaError_t launch_quantize_rows_e4m3(const bf16* in, long ld_in, int rows, int 
 
 cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream) {
   wait_timeout_selftest_kernel<<<1, 1, 0, stream>>>(limit_ns);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_exp2_fma_pipe(const float* x, float* y, long long n, cudaStream_t stream) {
-  if (n <= 0) return cudaSuccess;
-  long long blocks = (n / 2 + 255) / 256;
-  if (blocks < 1) blocks = 1;
-  if (blocks > 148LL * 8) blocks = 148LL * 8;
-  exp2_fma_pipe_kernel<<<(int)blocks, 256, 0, stream>>>(x, y, n);
   return cudaGetLastError();
 }
 

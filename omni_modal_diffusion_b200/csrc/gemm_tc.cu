@@ -113,8 +113,17 @@ __device__ __forceinline__ void epi_store_f32(const GemmEpilogue& e, uint32_t tb
       const int r = 4 * i + sub;
       if (m0 + r >= e.M) continue;
       const float4 w = *reinterpret_cast<const float4*>(stage + r * EPI_PITCH + 4 * (lane & 7));
-      float* dst = out + (long)(e.row_off + m0 + r) * e.ldo + col;
-      if (col + 4 <= e.N) {
+      const long off = (long)(e.row_off + m0 + r) * e.ldo + col;
+      float* dst = out + off;
+      if (e.euler) {
+        // one Euler step of the latent in out: out += dsigma * velocity
+        const float wv[4] = {w.x, w.y, w.z, w.w};
+        for (int k = 0; k < 4 && col + k < e.N; ++k) {
+          const float a = fmaf(e.dsigma, wv[k], dst[k]);
+          dst[k] = a;
+          if (e.out_bf16) e.out_bf16[off + k] = __float2bfloat16_rn(a);
+        }
+      } else if (col + 4 <= e.N) {
         *reinterpret_cast<float4*>(dst) = w;
       } else {
         const float wv[4] = {w.x, w.y, w.z, w.w};
@@ -339,7 +348,15 @@ __device__ __forceinline__ void epi_unpatch(const GemmEpilogue& e, uint32_t tb, 
         const int f = nc + jj;
         const int ph = f / (2 * C), pw = (f / C) % 2, ch = f % C;
         const long dst = (((long)t * (2 * e.Ht) + 2 * i + ph) * (2 * e.Wt) + 2 * j + pw) * C + ch;
-        static_cast<float*>(e.out)[dst] = v[jj];
+        float* o = static_cast<float*>(e.out) + dst;
+        if (e.euler) {
+          // one Euler step of the latent in out: out += dsigma * velocity
+          const float a = fmaf(e.dsigma, v[jj], *o);
+          *o = a;
+          if (e.out_bf16) e.out_bf16[dst] = __float2bfloat16_rn(a);
+        } else {
+          *o = v[jj];
+        }
       }
     }
   }

@@ -384,39 +384,60 @@ int h3_ffn_swiglu(const h3_dims* dims, const h3_ranges* ranges, float* x, const 
   return ok();
 }
 
-int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
-                   const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
-                   int C_audio, h3_bf16* hn, float* v_video, float* v_audio, void* stream) {
-  H3_TRACE();
-  H3_CHECK(check_dims(dims, __func__));
-  H3_CHECK(check_ranges(ranges, __func__));
+namespace {
+// The head (A10) and, with euler set, the Euler step (A11) in the head
+// GEMMs' epilogues.  Without euler: out_v / out_a receive the velocities.
+// With euler: out_v / out_a hold the latents, updated in place by
+// (sigma_next - sigma) * velocity, and out_v16 / out_a16 (nullable) receive
+// their bf16 copies.
+int head_impl(const char* fn, const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
+              const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio, int C_audio,
+              h3_bf16* hn, float* out_v, float* out_a, bool euler, float ds_v, float ds_a, h3_bf16* out_v16,
+              h3_bf16* out_a16, void* stream) {
+  H3_CHECK(check_dims(dims, fn));
+  H3_CHECK(check_ranges(ranges, fn));
   const int na = ranges->count[H3_AUDIO], nv = ranges->count[H3_VIDEO];
   if (T < 0 || (Hl & 1) || (Wl & 1) || (long)T * (Hl / 2) * (Wl / 2) != nv)
-    return fail(H3_ERR_SHAPE, "%s: count[VIDEO] != T*(Hl/2)*(Wl/2)", __func__);
-  if ((long)audio_channels * n_audio != na) return fail(H3_ERR_SHAPE, "%s: count[AUDIO] != channels*n_audio", __func__);
-  if (nv > 0 && (C_lat <= 0 || C_lat % 4)) return fail(H3_ERR_UNSUPPORTED, "%s: C_lat must be a multiple of 4", __func__);
-  if (na > 0 && (C_audio <= 0 || C_audio % 4)) return fail(H3_ERR_UNSUPPORTED, "%s: C_audio must be a multiple of 4", __func__);
-  H3_REQUIRE_PTR(x);
-  H3_REQUIRE_PTR(hn);
-  if (nv > 0) { H3_REQUIRE_PTR(W_vhead); H3_REQUIRE_PTR(v_video); }
-  if (na > 0) { H3_REQUIRE_PTR(W_ahead); H3_REQUIRE_PTR(v_audio); }
+    return fail(H3_ERR_SHAPE, "%s: count[VIDEO] != T*(Hl/2)*(Wl/2)", fn);
+  if ((long)audio_channels * n_audio != na) return fail(H3_ERR_SHAPE, "%s: count[AUDIO] != channels*n_audio", fn);
+  if (nv > 0 && (C_lat <= 0 || C_lat % 4)) return fail(H3_ERR_UNSUPPORTED, "%s: C_lat must be a multiple of 4", fn);
+  if (na > 0 && (C_audio <= 0 || C_audio % 4)) return fail(H3_ERR_UNSUPPORTED, "%s: C_audio must be a multiple of 4", fn);
+  if (!x) return fail(H3_ERR_NULL, "%s: argument 'x' is NULL", fn);
+  if (!aligned16(x)) return fail(H3_ERR_ALIGN, "%s: argument 'x' is not 16-byte aligned", fn);
+  if (!hn) return fail(H3_ERR_NULL, "%s: argument 'hn' is NULL", fn);
+  if (!aligned16(hn)) return fail(H3_ERR_ALIGN, "%s: argument 'hn' is not 16-byte aligned", fn);
+  const char* vname = euler ? "lat_video" : "v_video";
+  const char* aname = euler ? "lat_audio" : "v_audio";
+  if (nv > 0) {
+    if (!W_vhead || !out_v) return fail(H3_ERR_NULL, "%s: W_vhead or %s is NULL", fn, vname);
+    if (!aligned16(W_vhead) || !aligned16(out_v)) return fail(H3_ERR_ALIGN, "%s: W_vhead or %s not 16-byte aligned", fn, vname);
+    if (out_v16 && !aligned16(out_v16)) return fail(H3_ERR_ALIGN, "%s: lat_video_bf16 not 16-byte aligned", fn);
+  }
+  if (na > 0) {
+    if (!W_ahead || !out_a) return fail(H3_ERR_NULL, "%s: W_ahead or %s is NULL", fn, aname);
+    if (!aligned16(W_ahead) || !aligned16(out_a)) return fail(H3_ERR_ALIGN, "%s: W_ahead or %s not 16-byte aligned", fn, aname);
+    if (out_a16 && !aligned16(out_a16)) return fail(H3_ERR_ALIGN, "%s: lat_audio_bf16 not 16-byte aligned", fn);
+  }
   const int D = dims->D;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = launch_ln_modulate(x, nullptr, 0, ranges->start, ranges->count, ranges->L, ranges->L_pad, D,
                                      dims->eps_ln, reinterpret_cast<bf16*>(hn), st);
-  if (e != cudaSuccess) return cuda_fail(e, "h3_head_unpack: norm");
+  if (e != cudaSuccess) return cuda_fail(e, "head: norm");
   if (nv > 0) {
     const h3_bf16* A = hn + (size_t)ranges->start[H3_VIDEO] * D;
     GemmProblem p = gemm_base(A, D, nv, D, W_vhead, D, 4 * C_lat, (4 * C_lat + 255) / 256);
     p.epi.mode = EPI_UNPATCH;
     p.epi.M = nv;
     p.epi.N = 4 * C_lat;
-    p.epi.out = v_video;
+    p.epi.out = out_v;
     p.epi.Ht = Hl / 2;
     p.epi.Wt = Wl / 2;
     p.epi.C_lat = C_lat;
+    p.epi.euler = euler ? 1 : 0;
+    p.epi.dsigma = ds_v;
+    p.epi.out_bf16 = reinterpret_cast<bf16*>(out_v16);
     e = launch_gemm(p, st);
-    if (e != cudaSuccess) return cuda_fail(e, "h3_head_unpack: video head");
+    if (e != cudaSuccess) return cuda_fail(e, "head: video");
   }
   if (na > 0) {
     const h3_bf16* A = hn + (size_t)ranges->start[H3_AUDIO] * D;
@@ -425,10 +446,67 @@ int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x,
     p.epi.M = na;
     p.epi.N = C_audio;
     p.epi.ldo = C_audio;
-    p.epi.out = v_audio;
+    p.epi.out = out_a;
+    p.epi.euler = euler ? 1 : 0;
+    p.epi.dsigma = ds_a;
+    p.epi.out_bf16 = reinterpret_cast<bf16*>(out_a16);
     e = launch_gemm(p, st);
-    if (e != cudaSuccess) return cuda_fail(e, "h3_head_unpack: audio head");
+    if (e != cudaSuccess) return cuda_fail(e, "head: audio");
   }
+  return ok();
+}
+}  // namespace
+
+int h3_head_unpack(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
+                   const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
+                   int C_audio, h3_bf16* hn, float* v_video, float* v_audio, void* stream) {
+  H3_TRACE();
+  return head_impl(__func__, dims, ranges, x, W_vhead, W_ahead, T, Hl, Wl, C_lat, audio_channels, n_audio, C_audio,
+                   hn, v_video, v_audio, false, 0.f, 0.f, nullptr, nullptr, stream);
+}
+
+int h3_head_euler(const h3_dims* dims, const h3_ranges* ranges, const float* x, const h3_bf16* W_vhead,
+                  const h3_bf16* W_ahead, int T, int Hl, int Wl, int C_lat, int audio_channels, int n_audio,
+                  int C_audio, h3_bf16* hn, float* lat_video, float* lat_audio, float sigma_video,
+                  float sigma_video_next, float sigma_audio, float sigma_audio_next, h3_bf16* lat_video_bf16,
+                  h3_bf16* lat_audio_bf16, void* stream) {
+  H3_TRACE();
+  return head_impl(__func__, dims, ranges, x, W_vhead, W_ahead, T, Hl, Wl, C_lat, audio_channels, n_audio, C_audio,
+                   hn, lat_video, lat_audio, true, sigma_video_next - sigma_video, sigma_audio_next - sigma_audio,
+                   lat_video_bf16, lat_audio_bf16, stream);
+}
+
+size_t h3_adaln_workspace_bytes(int n, int c_dim) {
+  return (n > 0 && c_dim > 0) ? (size_t)n * (size_t)c_dim * 2 : 0;
+}
+
+int h3_adaln_modulation(const h3_dims* dims, const float* c, int n, int c_dim, const h3_bf16* W, h3_bf16* ws,
+                        float* mod, int64_t ld_mod, void* stream) {
+  H3_TRACE();
+  H3_CHECK(check_dims(dims, __func__));
+  if (n <= 0) return fail(H3_ERR_SHAPE, "%s: n must be positive (got %d)", __func__, n);
+  if (c_dim <= 0 || c_dim % 8 != 0)
+    return fail(H3_ERR_UNSUPPORTED, "%s: c_dim must be a positive multiple of 8 (got %d)", __func__, c_dim);
+  H3_REQUIRE_PTR(c);
+  H3_REQUIRE_PTR(W);
+  H3_REQUIRE_PTR(ws);
+  H3_REQUIRE_PTR(mod);
+  const int N = 18 * dims->D;
+  if (ld_mod == 0) ld_mod = N;
+  if (ld_mod < N || ld_mod % 4 != 0)
+    return fail(H3_ERR_SHAPE, "%s: ld_mod must be 0 or a multiple of 4 of at least 18 D (got %lld)", __func__,
+                (long long)ld_mod);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_silu_bf16(c, (long long)n * c_dim, reinterpret_cast<bf16*>(ws), st);
+  if (e != cudaSuccess) return cuda_fail(e, "h3_adaln_modulation: silu");
+  GemmProblem p = gemm_base(ws, c_dim, n, c_dim, W, c_dim, N, (N + 255) / 256);
+  p.epi.mode = EPI_STORE_F32;
+  p.epi.M = n;
+  p.epi.N = N;
+  p.epi.ldo = ld_mod;
+  p.epi.out = mod;
+  e = launch_gemm(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "h3_adaln_modulation: linear");
   return ok();
 }
 
@@ -514,17 +592,6 @@ int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, con
   H3_CHECK(h3_gated_residual(dims, ranges, x, buf->o, w->Wo, mod, H3_MSA, stream));
   H3_CHECK(h3_adaln_norm_modulate(dims, ranges, x, mod, H3_MLP, buf->xm, stream));
   H3_CHECK(h3_ffn_swiglu(dims, ranges, x, buf->xm, w->Wgu, w->Wd, mod, buf->ws, stream));
-  return ok();
-}
-
-int h3_exp2_fma_pipe(const float* x, float* y, int64_t n, void* stream) {
-  H3_TRACE();
-  if (n < 0) return fail(H3_ERR_SHAPE, "h3_exp2_fma_pipe: n < 0");
-  if (n == 0) return ok();
-  H3_REQUIRE_PTR(x);
-  H3_REQUIRE_PTR(y);
-  cudaError_t e = launch_exp2_fma_pipe(x, y, (long long)n, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "h3_exp2_fma_pipe");
   return ok();
 }
 

@@ -45,6 +45,13 @@ struct GemmEpilogue {
   int qk_e4m3;
   // EPI_UNPATCH: token grid (T, Ht, Wt), latent channels
   int Ht, Wt, C_lat;
+  // EPI_STORE_F32 / EPI_UNPATCH with euler != 0: out holds a latent that
+  // takes one Euler step in place, out[i] = out[i] + dsigma * acc (acc is the
+  // velocity), and out_bf16 (when set, same layout) receives bf16(out[i])
+  // after the update
+  int euler;
+  float dsigma;
+  bf16* out_bf16;
   // e4m3 operands: acc[m][n] *= a_scale[m] * b_scale[n] before the epilogue
   // (a_scale per A row, b_scale per B row); null for bf16 operands.  Set by
   // launch_gemm from GemmProblem.
@@ -116,10 +123,10 @@ cudaError_t launch_ln_modulate_e4m3(const float* x, const float* mod, int branch
 cudaError_t launch_quantize_rows_e4m3(const bf16* in, long ld_in, int rows, int cols, uint8_t* q, long ld_q,
                                       float* scale, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(unsigned long long limit_ns, cudaStream_t stream);
-cudaError_t launch_exp2_fma_pipe(const float* x, float* y, long long n, cudaStream_t stream);
 cudaError_t launch_euler_bf16(float* lat, const float* vel, long long n, float dsigma, bf16* out,
                               cudaStream_t stream);
 cudaError_t launch_euler(float* lat, const float* vel, long long n, float dsigma, cudaStream_t stream);
+cudaError_t launch_silu_bf16(const float* c, long long n, bf16* a, cudaStream_t stream);
 
 int num_sms();
 

@@ -411,28 +411,43 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// 2^x for two lanes on the FMA pipe, x in [-125, 64] (clamped below): x = j + f with
-// j = rint(x) (adding 1.5 * 2^23 leaves j in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f from a cubic fitted for this library by Remez
-// exchange on the relative error (max relative error 7.5e-5, far below the
-// bf16 rounding that follows); 2^j is added to the exponent field
-// (the 1.5 * 2^23 bias shifts out of the 32-bit word when moved left by 23).
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t t = f2_add(x, magic);
-  const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
+// a * b + c rounded once, the result clamped to [0, 1]
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe for a pair of lanes, without the MUFU unit; x is given
+// as x = s * a + b with a = k / 252, b = (125 + c) / 252 (so x = k s + c).
+//   u = sat(s a + b) in [0, 1] puts x' = 252 u - 125 in [-125, 127]: the
+//       clamp costs no extra instruction, masks nothing that matters (2^-125
+//       is below every sum it joins; 2^127 still fails any overflow check);
+//   t = 252 u + (1.5 * 2^23 - 125) rounds 252 u to the integer R in the low
+//       mantissa bits, so bits(t) = bits(1.5 * 2^23) + j with j = R - 125;
+//   f = 252 u - R in [-1/2, 1/2];
+//   2^f from a cubic fitted for this library by Remez exchange on the
+//       relative error over [-1/2, 1/2] (max relative error 7.5e-5, far below
+//       the bf16 rounding of P that follows), in [0.707, 1.415];
+//   2^x' = 2^f with j added to its exponent field: bits(t) << 23 is j << 23
+//       (the bias bits shift out of the word), and the exponent stays in
+//       [1, 254] for j in [-125, 127].
+// Returns the two results as f32x2.
+__device__ __forceinline__ uint64_t exp2_fma2(float s0, float s1, float a, float b) {
+  const uint64_t u = f2_pack(fma_sat(s0, a, b), fma_sat(s1, a, b));
+  const uint64_t k252 = f2_pack(252.0f, 252.0f);
+  const float kShift = 12582787.0f;  // 1.5 * 2^23 - 125
+  const uint64_t t = f2_fma(u, k252, f2_pack(kShift, kShift));
+  const uint64_t nR = f2_fma(t, f2_pack(-1.0f, -1.0f), f2_pack(kShift, kShift));  // -R, exact
+  const uint64_t f = f2_fma(u, k252, nR);
   uint64_t p = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.2426111251f, 0.2426111251f));
   p = f2_fma(p, f, f2_pack(0.6932609677f, 0.6932609677f));
   p = f2_fma(p, f, f2_pack(0.9999280572f, 0.9999280572f));
   float p0, p1, t0, t1;
   f2_unpack(p, p0, p1);
   f2_unpack(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
 // Two fp32 -> two e4m3 codes, round to nearest even, saturating to +-448

@@ -24,8 +24,10 @@ H3_QK_E4M3 = 2  # q, k as e4m3 codes between the e4m3 QKV call and attention
 EXPORTS = (
     "h3_last_error", "h3_version", "h3_make_ranges", "h3_sigma_schedule", "h3_embed_pack",
     "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention", "h3_gated_residual",
-    "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step", "h3_device_status",
-    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_exp2_fma_pipe", "h3_block_forward",
+    "h3_ffn_workspace_bytes", "h3_ffn_swiglu", "h3_head_unpack", "h3_head_euler", "h3_euler_step",
+    "h3_adaln_workspace_bytes", "h3_adaln_modulation",
+    "h3_device_status",
+    "h3_set_wait_limit_ns", "h3_ffn_swiglu_noalloc", "h3_block_forward",
     "h3_euler_step_bf16", "h3_selftest_wait_timeout",
     "h3_quantize_rows_e4m3", "h3_adaln_norm_modulate_e4m3", "h3_qkv_qknorm_mrope_e4m3", "h3_gated_residual_e4m3",
     "h3_ffn_e4m3_workspace_bytes", "h3_ffn_swiglu_e4m3", "h3_block_forward_e4m3",
@@ -108,8 +110,11 @@ def lib() -> ctypes.CDLL:
             "h3_ffn_swiglu": (ci, [pd, pr, vp, vp, vp, vp, vp, vp, vp]),
             "h3_ffn_swiglu_noalloc": (ci, [pd, pr, vp, vp, vp, vp, vp, vp]),
             "h3_head_unpack": (ci, [pd, pr, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp]),
+            "h3_head_euler": (ci, [pd, pr, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, cf, cf, cf, cf, vp, vp,
+                                   vp]),
+            "h3_adaln_workspace_bytes": (ctypes.c_size_t, [ci, ci]),
+            "h3_adaln_modulation": (ci, [pd, vp, ci, ci, vp, vp, vp, ctypes.c_int64, vp]),
             "h3_euler_step": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp]),
-            "h3_exp2_fma_pipe": (ci, [vp, vp, ctypes.c_int64, vp]),
             "h3_euler_step_bf16": (ci, [vp, vp, ctypes.c_int64, cf, cf, vp, vp]),
             "h3_block_forward": (ci, [pd, pr, vp, vp, vp, ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockBuffers),
                                       ci, vp]),
@@ -242,6 +247,40 @@ def h3_head_unpack(dims, ranges, x, W_vhead, W_ahead, video_shape, audio_shape, 
                                 _ptr(v_audio, F32, "v_audio"), _stream(stream)))
 
 
+def h3_head_euler(dims, ranges, x, W_vhead, W_ahead, video_shape, audio_shape, hn, lat_video, lat_audio,
+                  sig_video, sig_audio, lat_video_bf16=None, lat_audio_bf16=None, stream=None):
+    """sig_video, sig_audio: (sigma, sigma_next) of each modality's schedule."""
+    T, Hl, Wl, C_lat = video_shape
+    ch, n_a, C_a = audio_shape
+    _check(lib().h3_head_euler(ctypes.byref(dims), ctypes.byref(ranges), _ptr(x, F32, "x"),
+                               _ptr(W_vhead, BF16, "W_vhead"), _ptr(W_ahead, BF16, "W_ahead"), T, Hl, Wl, C_lat, ch,
+                               n_a, C_a, _ptr(hn, BF16, "hn"), _ptr(lat_video, F32, "lat_video"),
+                               _ptr(lat_audio, F32, "lat_audio"), float(sig_video[0]), float(sig_video[1]),
+                               float(sig_audio[0]), float(sig_audio[1]), _ptr(lat_video_bf16, BF16, "lat_video_bf16"),
+                               _ptr(lat_audio_bf16, BF16, "lat_audio_bf16"), _stream(stream)))
+
+
+def h3_adaln_workspace_bytes(n: int, c_dim: int) -> int:
+    return int(lib().h3_adaln_workspace_bytes(n, c_dim))
+
+
+def h3_adaln_modulation(dims, c, W, ws, mod, stream=None):
+    """mod = W SiLU(c) for c [n][c_dim] fp32, W [18D][c_dim] bf16; ws: bf16
+    scratch of n * c_dim elements.  mod: a contiguous [n][3][6][D] fp32
+    tensor, or a view whose rows (first index) are apart by its stride, e.g.
+    cache[:, b] of a [step][block][3][6][D] cache."""
+    n, c_dim = c.shape
+    if ws.numel() * ws.element_size() < h3_adaln_workspace_bytes(n, c_dim):
+        raise ValueError("workspace too small")
+    if not (isinstance(mod, torch.Tensor) and mod.is_cuda and mod.dtype == F32):
+        raise TypeError("mod must be a float32 CUDA tensor")
+    if mod.shape[0] != n or mod[0].numel() != 18 * dims.D or (n > 1 and not mod[0].is_contiguous()):
+        raise ValueError("mod must be [n][3][6][D] with contiguous rows")
+    ld = mod.stride(0) if n > 1 else 18 * dims.D
+    _check(lib().h3_adaln_modulation(ctypes.byref(dims), _ptr(c, F32, "c"), n, c_dim, _ptr(W, BF16, "W"),
+                                     _ptr(ws, BF16, "ws"), ctypes.c_void_p(mod.data_ptr()), ld, _stream(stream)))
+
+
 def h3_euler_step(lat, vel, sigma: float, sigma_next: float, stream=None):
     if lat.numel() != vel.numel():
         raise ValueError("lat and vel sizes differ")
@@ -270,10 +309,6 @@ def h3_euler_step_bf16(lat, vel, sigma: float, sigma_next: float, lat_bf16, stre
         raise ValueError("lat, vel and lat_bf16 sizes differ")
     _check(lib().h3_euler_step_bf16(_ptr(lat, F32, "lat"), _ptr(vel, F32, "vel"), lat.numel(), sigma, sigma_next,
                                     _ptr(lat_bf16, BF16, "lat_bf16"), _stream(stream)))
-
-
-def h3_exp2_fma_pipe(x, y, stream=None):
-    _check(lib().h3_exp2_fma_pipe(_ptr(x, F32, "x"), _ptr(y, F32, "y"), x.numel(), _stream(stream)))
 
 
 def h3_device_status(stream=None) -> int:

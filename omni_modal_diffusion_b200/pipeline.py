@@ -133,12 +133,20 @@ class H3BlockStep:
         h3.h3_euler_step(lat_video, self.v_video, sig_video[0], sig_video[1], stream=stream)
         h3.h3_euler_step(lat_audio, self.v_audio, sig_audio[0], sig_audio[1], stream=stream)
 
+    def head_euler(self, lat_video, lat_audio, sig_video, sig_audio, video_bf16=None, audio_bf16=None, stream=None):
+        """Head and Euler step in one call (h3_head_euler): the latents move
+        by (sigma_next - sigma) * velocity in the head GEMMs' epilogues; the
+        bf16 copies, when given, receive the updated latents."""
+        w = self.w
+        h3.h3_head_euler(self.dims, self.ranges, self.x, self.W["W_vhead"], self.W["W_ahead"],
+                         (w.T_lat, w.H_lat, w.W_lat, w.C_lat), (w.audio_channels, w.n_audio, w.C_audio), self.hn,
+                         lat_video, lat_audio, sig_video, sig_audio, video_bf16, audio_bf16, stream=stream)
+
     def step(self, text, video, audio, mod, lat_video, lat_audio, sig_video, sig_audio, stream=None):
-        """The whole hot path once: pack/project, one block, head, Euler x2."""
+        """The whole hot path once: pack/project, one block, head + Euler."""
         self.embed(text, video, audio, stream)
         self.block(mod, stream=stream)
-        self.head(stream)
-        self.euler(lat_video, lat_audio, sig_video, sig_audio, stream)
+        self.head_euler(lat_video, lat_audio, sig_video, sig_audio, stream=stream)
 
     # kernels launched by one step (for the launch count the bench reports)
     def launches_per_step(self, e4m3: bool = False) -> int:
@@ -146,8 +154,9 @@ class H3BlockStep:
         embed = (1 if r.count[2] > 0 else 0) + 1 + (1 if r.L_pad > r.L else 0) + sum(1 for c in r.count if c > 0)
         # LN, QKV, attention, [quantise o,] out-projection, LN, FFN (2 GEMMs [+ quantise h])
         block = 1 + 1 + 1 + 1 + 1 + 2 + (2 if e4m3 else 0)
+        # head + Euler: LN, video head GEMM, audio head GEMM (Euler in their epilogues)
         head = 1 + (1 if r.count[2] > 0 else 0) + (1 if r.count[1] > 0 else 0)
-        return embed + block + head + 2
+        return embed + block + head
 
 
 class H3Sampler:
@@ -156,9 +165,9 @@ class H3Sampler:
     Euler update of the generation targets only; text is a fixed condition).
 
     Per denoise step: pack + project the bf16 latents, n_layers blocks
-    (h3_block_forward, modulation [step][layer][3][6][D]), head, then one
-    Euler step per modality that also writes the bf16 latent for the next
-    step.  Orchestration only: every step runs in the library's kernels.
+    (h3_block_forward, modulation [step][layer][3][6][D]), then the head with
+    each modality's Euler step in its epilogue (h3_head_euler), which also
+    writes the bf16 latents for the next step.  Orchestration only: every step runs in the library's kernels.
 
     e4m3=True runs the blocks with their four GEMMs on e4m3 operands
     (h3_block_forward_e4m3): each block's weights are quantised once on the
@@ -199,9 +208,7 @@ class H3Sampler:
         for b in range(self.n_layers):
             forward(st.dims, st.ranges, st.x, mod_all[s, b], st.pos, self.blocks[b], self.bufs, flags=self.flags,
                     stream=stream)
-        st.head(stream)
-        h3.h3_euler_step_bf16(lat_video, st.v_video, sv[s], sv[s + 1], video_bf16, stream=stream)
-        h3.h3_euler_step_bf16(lat_audio, st.v_audio, sa[s], sa[s + 1], audio_bf16, stream=stream)
+        st.head_euler(lat_video, lat_audio, (sv[s], sv[s + 1]), (sa[s], sa[s + 1]), video_bf16, audio_bf16, stream)
 
     def run(self, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, n_steps: int, stream=None,
             start_step: int = 0, end_step: int | None = None):
@@ -214,6 +221,22 @@ class H3Sampler:
         sa = h3.h3_sigma_schedule(n_steps, self.shifts[1])
         for s in range(start_step, n_steps if end_step is None else end_step):
             self.step(s, text, lat_video, lat_audio, video_bf16, audio_bf16, mod_all, sv, sa, stream)
+
+    def modulation_cache(self, c_steps, adaln_weights: list, stream=None):
+        """The modulation cache [n_steps][n_layers][3][6][D] fp32 that run()
+        reads, from each step's conditioning vector (c_steps [n_steps][c_dim]
+        fp32) and each block's AdaLN producer weight ([18 D][c_dim] bf16),
+        one h3_adaln_modulation call per block writing its column of the
+        cache."""
+        st = self.st
+        n_steps, c_dim = c_steps.shape
+        if len(adaln_weights) != self.n_layers:
+            raise ValueError("one AdaLN weight per block")
+        mod_all = torch.empty(n_steps, self.n_layers, 3, 6, st.w.D, dtype=torch.float32, device=st.device)
+        ws = torch.empty(h3.h3_adaln_workspace_bytes(n_steps, c_dim) // 2, dtype=torch.bfloat16, device=st.device)
+        for b, Wb in enumerate(adaln_weights):
+            h3.h3_adaln_modulation(st.dims, c_steps, Wb, ws, mod_all[:, b], stream=stream)
+        return mod_all
 
     # ---------------------------------------------------------- checkpoint / resume
     @staticmethod
@@ -237,4 +260,4 @@ class H3Sampler:
     def launches_per_step(self) -> int:
         st = self.st
         per_block = 9 if self.e4m3 else 7
-        return st.launches_per_step() - 2 - 7 + per_block * self.n_layers + 2
+        return st.launches_per_step() - 7 + per_block * self.n_layers

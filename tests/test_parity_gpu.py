@@ -7,6 +7,7 @@ latents and features in, oracle recomputes everything).  Integer, byte and
 index work is compared bit-exactly; floating point within the block tolerance
 of parity_util.check_close unless a test states a tighter bound.
 """
+import dataclasses
 import functools
 
 import numpy as np
@@ -191,6 +192,54 @@ def test_head_unpack_seeded(w):
                            w.n_audio)
     check_close(to_np(vv), rv, "video head", 3e-2, 3e-3)       # bf16 normalised input (see LN test)
     check_close(to_np(va), ra, "audio head", 3e-2, 3e-3)
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+def test_head_euler_fused(w):
+    """h3_head_euler (the Euler step in the head GEMMs' epilogues) equals
+    h3_head_unpack followed by h3_euler_step on each latent bit for bit,
+    writes the bf16 copies of the updated latents, and matches the oracle's
+    head + Euler step (each modality on its own shifted schedule)."""
+    inp = _inputs(w)
+    r, _ = oracle_ranges_and_pos(w)
+    L, Lp = r["L"], r["L_pad"]
+    rng = np.random.default_rng(83 + w.index)
+    x = _rows_stream(w, rng, L, Lp, w.D)
+    lv0 = rng.standard_normal((w.T_lat, w.H_lat, w.W_lat, w.C_lat)).astype(np.float32)
+    la0 = rng.standard_normal((w.audio_channels, w.n_audio, w.C_audio)).astype(np.float32)
+    d, rg = h3.make_dims(w.D, w.H, w.F), h3.h3_make_ranges(*r["count"])
+    sv = h3.h3_sigma_schedule(8, 12.0)
+    sa = h3.h3_sigma_schedule(8, 3.0)
+    Wv, Wa = to_dev_bf16(inp["W_vhead"], DEV), to_dev_bf16(inp["W_ahead"], DEV)
+    hn = torch.empty(Lp, w.D, dtype=torch.bfloat16, device=DEV)
+    shapes = ((w.T_lat, w.H_lat, w.W_lat, w.C_lat), (w.audio_channels, w.n_audio, w.C_audio))
+    for s in (0, 5):
+        lv, la = _f32(lv0), _f32(la0)
+        lv16 = torch.full(lv.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+        la16 = torch.full(la.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+        h3.h3_head_euler(d, rg, _f32(x), Wv, Wa, *shapes, hn, lv, la, (sv[s], sv[s + 1]), (sa[s], sa[s + 1]),
+                         lv16, la16)
+        # unfused reference path through the library
+        vv, va = torch.empty_like(lv), torch.empty_like(la)
+        h3.h3_head_unpack(d, rg, _f32(x), Wv, Wa, *shapes, hn, vv, va)
+        lv_ref, la_ref = _f32(lv0), _f32(la0)
+        h3.h3_euler_step(lv_ref, vv, sv[s], sv[s + 1])
+        h3.h3_euler_step(la_ref, va, sa[s], sa[s + 1])
+        torch.cuda.synchronize()
+        assert torch.equal(lv, lv_ref) and torch.equal(la, la_ref)
+        assert torch.equal(lv16, lv.to(torch.bfloat16)) and torch.equal(la16, la.to(torch.bfloat16))
+        rv, ra = O.head_unpack(x[:L], r, inp["W_vhead"], inp["W_ahead"], w.T_lat, w.H_lat, w.W_lat,
+                               w.audio_channels, w.n_audio)
+        ov = O.euler_step(lv0, rv, np.float64(np.float32(sv[s])), np.float64(np.float32(sv[s + 1])))
+        oa = O.euler_step(la0, ra, np.float64(np.float32(sa[s])), np.float64(np.float32(sa[s + 1])))
+        # the latent change (the head's contribution) at the head's bound
+        check_close(to_np(lv) - lv0, ov - lv0, f"video latent change, step {s}", 3e-2, 3e-3)
+        check_close(to_np(la) - la0, oa - la0, f"audio latent change, step {s}", 3e-2, 3e-3)
+    # without bf16 copies (NULL) the latents are the same
+    lv, la = _f32(lv0), _f32(la0)
+    h3.h3_head_euler(d, rg, _f32(x), Wv, Wa, *shapes, hn, lv, la, (sv[5], sv[6]), (sa[5], sa[6]))
+    torch.cuda.synchronize()
+    assert torch.equal(lv, lv_ref) and torch.equal(la, la_ref)
 
 
 def test_euler_and_schedule_seeded():
@@ -394,6 +443,41 @@ def test_full_length_attention_sampled_rows(L, H):
         assert float(o[L:].float().abs().max()) == 0.0
 
 
+# The 15 s workload's token layout (512 text, 2 x 600 audio, 91 x 24 x 56
+# video tokens: L = 124,016, L_pad = 124,032, 969 query tiles, so the last
+# attention CTA holds one tile) at the tiny widths, so that the oracle can
+# follow sampled rows through the whole block at that length.
+LONG_TINY = dataclasses.replace(S.WORKLOADS["768x1792_15s"], name="768x1792_15s_tiny_width", index=30, D=320, H=4,
+                                F=896, D_text=256)
+
+
+def test_long_sequence_block_tiny_width_sampled_rows():
+    """The whole block (embed, LN + modulate, QKV + RMSNorm + RoPE,
+    attention over 124,016 tokens, gated out-projection, SwiGLU FFN) at the
+    longest packed length with the tiny widths; the oracle follows sampled
+    rows (K and V of every token, per head), including the first and last
+    rows of every modality range and rows of the last, single-tile CTA."""
+    w = LONG_TINY
+    inp, st, text, video, audio, mod = _setup(w)
+    r, pos = oracle_ranges_and_pos(w)
+    L = r["L"]
+    assert L == 124016 and r["L_pad"] // 128 % 2 == 1
+    st.embed(text, video, audio)
+    x0_gpu = to_np(st.x[:L])
+    st.block(mod)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    edges = [s + c - 1 for s, c in zip(r["start"], r["count"])] + list(r["start"]) + [L - 128, L - 3]
+    rows = np.unique(np.concatenate([_sample_rows(L, 24, seed=1792), edges]))
+    x0 = O.embed(inp["text"], inp["video"], inp["audio"], inp["W_text"], inp["W_vid"], inp["W_aud"], r)
+    check_close(x0_gpu[rows], x0[rows], "embedded rows", 1e-4, 1e-5)
+    ref, _ = O.block_forward_rows(x0, inp["mod"], r, pos, rows, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"],
+                                  inp["Wgu"], inp["Wd"], w.H)
+    x2 = to_np(st.x[torch.from_numpy(rows).to(DEV)])
+    check_close(x2, ref, "124k-token block output rows")
+    check_close(x2 - x0[rows], ref - x0[rows], "124k-token block delta rows", max_rel_rms=5e-2)
+
+
 def test_full_length_qkv_sampled_rows():
     """QKV + Q/K RMSNorm + RoPE at the longest packed length (124,016 tokens,
     969 row tiles), sampled rows, real positions of that workload."""
@@ -419,21 +503,3 @@ def test_full_length_qkv_sampled_rows():
 
 def test_device_status_clean_after_work():
     assert h3.h3_device_status() == 0
-
-
-def test_exp2_fma_pipe_error_bound():
-    """The softmax's FMA-pipe exponential stays within its stated 7.5e-5
-    relative error of 2^x over the range the softmax feeds it (x <= 8 after
-    the lazy max; down to the -125 clamp), and matches the clamp below."""
-    x = np.concatenate([np.linspace(-125.0, 64.0, 2_000_001), np.arange(-125, 64, dtype=np.float64) + 0.5,
-                        np.arange(-125, 65, dtype=np.float64)]).astype(np.float32)
-    y = torch.empty(len(x), device=DEV)
-    h3.h3_exp2_fma_pipe(_f32(x), y)
-    got = to_np(y)
-    ref = np.exp2(x.astype(np.float64))
-    rel = np.abs(got / ref - 1.0)
-    assert rel.max() <= 7.6e-5, rel.max()
-    z = torch.empty(3, device=DEV)
-    h3.h3_exp2_fma_pipe(_f32(np.array([-200.0, -1e30, -125.0], np.float32)), z)
-    zz = to_np(z)
-    assert np.allclose(zz, 2.0 ** -125, rtol=1e-4)
