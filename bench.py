@@ -2,21 +2,34 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
+The default workload is the longest single-GPU one, 768x1792_15s (124,016
+packed tokens: 21:9 768x1792, 15 s at 24 fps, stereo audio, 512 text tokens);
+768sq_2s and 768x1344_5s are the same line with --workload.
 One step = the whole hot path once over one packed sequence: patchify + pack +
 per-modality input projections, one full-width block (LN+modulate, QKV with
 Q/K RMSNorm + 3-D RoPE, attention, gated out-projection, LN+modulate, gated
-SwiGLU FFN), the output head and the two Euler updates (video, audio).
+SwiGLU FFN), and the output head with the two Euler updates (video, audio)
+in its GEMM epilogues (h3_head_euler).
 Every rank processes its own sequence (independent requests, no collective):
 weak scaling, value = tokens of all ranks / max-over-ranks time.
 
 --impl reference times the float64 CPU oracle on a bounded sample of the same
 workload (the reference arm of this comparison; it is not tuned).
 
+--sp times sequence parallelism instead: one sequence split over the job's
+ranks (strong scaling; its own line).
 Separate lines (one GPU each, not the headline): --e4m3 (the block's four
 GEMMs on e4m3 operands; with --qk-e4m3 also attention's Q K^T on e4m3
 codes), --sampler (the 50-block, 8-step layered sampler on 768x1344_5s;
 combinable with --e4m3 [--qk-e4m3]), --only CALL (one C-ABI call alone, for
-ncu captures; prints a timing line, not the JSON contract line).
+ncu captures; prints a timing line, not the JSON contract line; --heads H
+runs it with H heads instead of the workload's, for captures that must stay
+small).
+
+Roofline peaks: a timed region of a second or more runs under the 1 kW power
+cap, so its fractions are against the measured sustained bf16 matmul figure;
+a shorter one against the measured burst figure.  Every kernel also carries
+its fraction of the burst figure and of the 2.25 PFLOP/s dense bf16 spec.
 """
 from __future__ import annotations
 
@@ -36,7 +49,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "packed tokens/s per Omni block (bf16, 1×B200) & % of dense bf16 tensor peak"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "768sq_2s"
+DEFAULT_WORKLOAD = "768x1792_15s"
+BF16_SPEC_TFLOPS = 2250.0
 
 
 def _peaks():
@@ -64,9 +78,13 @@ def bytes_per_call(w, L, Lp):
     """Algorithmic HBM bytes of the memory-bound calls."""
     D = w.D
     n_lat = w.T_lat * w.H_lat * w.W_lat * w.C_lat + w.audio_channels * w.n_audio * w.C_audio
+    n_gen = w.audio_channels * w.n_audio + w.T_lat * (w.H_lat // 2) * (w.W_lat // 2)   # audio + video rows
     return {
         "h3_adaln_norm_modulate": L * (4 * D + 2 * D) + (Lp - L) * 2 * D,
-        "h3_euler_step": 12 * n_lat,
+        # head + Euler: LN of the generated rows (read x fp32, write hn bf16),
+        # the head GEMMs read hn and their weights, each latent element is read
+        # and written once (fp32); the velocity never goes to memory
+        "h3_head_euler": n_gen * (4 * D + 2 * D) + n_gen * 2 * D + (4 * w.C_lat + w.C_audio) * D * 2 + 8 * n_lat,
     }
 
 
@@ -82,6 +100,21 @@ TRAFFIC = {
     # one attention launch
     ("768sq_2s", "attention_tc_kernel"): 0.4379e9,
 }
+
+
+def peak_for_region(peaks, region_s):
+    """(peak TFLOP/s, its name) for a timed region of region_s seconds: the
+    sustained figure once the region runs long enough to settle under the
+    power cap (>= 1 s), else the burst figure."""
+    if region_s >= 1.0:
+        return peaks["bf16_tflops_sustained"], f"bf16 sustained, of {peaks['source']} (timed region {region_s:.1f} s)"
+    return peaks["bf16_tflops"], f"bf16 burst, of {peaks['source']} (timed region {region_s:.2f} s)"
+
+
+def kernel_entry(ms, launches, tflops, peak_tf, peaks, traffic):
+    return {"ms_per_step": round(ms, 4), "launches_per_step": launches, "tflops": round(tflops, 1),
+            "frac": round(tflops / peak_tf, 4), "frac_of_burst": round(tflops / peaks["bf16_tflops"], 4),
+            "frac_of_spec_2250": round(tflops / BF16_SPEC_TFLOPS, 4), "traffic_per_launch": traffic}
 
 
 class ClockSampler:
@@ -192,7 +225,7 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream(dev)
 
     calls = ["h3_embed_pack", "h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
-             "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu", "h3_head_unpack", "h3_euler_step"]
+             "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu", "h3_head_euler"]
 
     def step(i, ev=None):
         s = i % 8
@@ -207,8 +240,7 @@ def run_ours(args, w):
         mark(4, 0); h3.h3_gated_residual(d, r, st.x, st.o, st.W["Wo"], mod, h3.H3_MSA); mark(4, 1)
         mark(5, 0); h3.h3_adaln_norm_modulate(d, r, st.x, mod, h3.H3_MLP, st.xm); mark(5, 1)
         mark(6, 0); h3.h3_ffn_swiglu(d, r, st.x, st.xm, st.W["Wgu"], st.W["Wd"], mod, st.ws); mark(6, 1)
-        mark(7, 0); st.head(); mark(7, 1)
-        mark(8, 0); st.euler(lat_v, lat_a, (sv[s], sv[s + 1]), (sa[s], sa[s + 1])); mark(8, 1)
+        mark(7, 0); st.head_euler(lat_v, lat_a, (sv[s], sv[s + 1]), (sa[s], sa[s + 1])); mark(7, 1)
 
     def barrier():
         if world > 1:
@@ -315,7 +347,7 @@ def run_ours(args, w):
     fl = flops_per_call(w, L)
     by = bytes_per_call(w, L, Lp)
     tensor_calls = {c: fl[c] / (per_call[c] / 1e3) / 1e12 for c in fl}
-    peak_tf = peaks["bf16_tflops_sustained"]
+    peak_tf, peak_kind = peak_for_region(peaks, ms_total / 1e3)
     # Kernels: the tcgen05 GEMM (gemm_tc2_kernel, CTA pairs, for QKV and the
     # out-projection; gemm_tc_kernel for the FFN's gate/up and down) runs the
     # block's four GEMM launches (the embed/head launches add < 0.4% of its
@@ -324,20 +356,16 @@ def run_ours(args, w):
     gemm_ms = sum(per_call[c] for c in gemm_calls)
     gemm_tf = sum(fl[c] for c in gemm_calls) / (gemm_ms / 1e3) / 1e12
     attn_tf = tensor_calls["h3_attention"]
-    kernels = {"gemm_tc_kernel": {"ms_per_step": round(gemm_ms, 4), "launches_per_step": 4,
-                                  "tflops": round(gemm_tf, 1), "frac": round(gemm_tf / peak_tf, 4),
-                                  "traffic_per_launch": TRAFFIC.get((w.name, "gemm_tc_kernel"))},
-               "attention_tc_kernel": {"ms_per_step": round(per_call["h3_attention"], 4), "launches_per_step": 1,
-                                       "tflops": round(attn_tf, 1), "frac": round(attn_tf / peak_tf, 4),
-                                       "traffic_per_launch": TRAFFIC.get((w.name, "attention_tc_kernel"))}}
+    kernels = {"gemm_tc_kernel": kernel_entry(gemm_ms, 4, gemm_tf, peak_tf, peaks,
+                                              TRAFFIC.get((w.name, "gemm_tc_kernel"))),
+               "attention_tc_kernel": kernel_entry(per_call["h3_attention"], 1, attn_tf, peak_tf, peaks,
+                                                   TRAFFIC.get((w.name, "attention_tc_kernel")))}
     dominant = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     block_flops = sum(fl.values())
     block_ms = sum(per_call[c] for c in ("h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
                                          "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu"))
     ln_gbs = by["h3_adaln_norm_modulate"] / (per_call["h3_adaln_norm_modulate"] / 1e3) / 1e9
-    # two launches (video and audio latents); the latents were just written
-    # by the head, so at this size they are read from L2
-    euler_gbs = by["h3_euler_step"] / (per_call["h3_euler_step"] / 1e3) / 1e9
+    head_gbs = by["h3_head_euler"] / (per_call["h3_head_euler"] / 1e3) / 1e9
     launches = st.launches_per_step()
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -352,17 +380,19 @@ def run_ours(args, w):
         "roofline": {"bound": "tensor", "kernel": dominant,
                      "achieved": kernels[dominant]["tflops"],
                      "peak": peak_tf, "unit": "TFLOP/s", "frac": kernels[dominant]["frac"],
-                     "peak_kind": f"bf16 sustained, of measured ({peaks['source']})",
+                     "peak_kind": peak_kind, "frac_of_burst": kernels[dominant]["frac_of_burst"],
+                     "frac_of_spec_2250": kernels[dominant]["frac_of_spec_2250"],
                      "traffic": TRAFFIC.get((w.name, dominant))},
         "kernels": kernels,
         "block": {"tflops": round(block_flops / (block_ms / 1e3) / 1e12, 1),
-                  "frac_of_bf16_sustained": round(block_flops / (block_ms / 1e3) / 1e12 / peak_tf, 4),
-                  "frac_of_bf16_spec_2250": round(block_flops / (block_ms / 1e3) / 1e12 / 2250.0, 4),
+                  "frac": round(block_flops / (block_ms / 1e3) / 1e12 / peak_tf, 4),
+                  "frac_of_burst": round(block_flops / (block_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+                  "frac_of_spec_2250": round(block_flops / (block_ms / 1e3) / 1e12 / BF16_SPEC_TFLOPS, 4),
                   "ms": round(block_ms, 4)},
         "per_call_ms": {c: round(v, 4) for c, v in per_call.items()},
         "per_call_tflops": {c: round(v, 1) for c, v in tensor_calls.items()},
         "ln_modulate_gbs": round(ln_gbs, 1), "ln_modulate_frac_hbm": round(ln_gbs / peaks["hbm_gbs"], 4),
-        "euler_gbs": round(euler_gbs, 1), "euler_frac_hbm": round(euler_gbs / peaks["hbm_gbs"], 4),
+        "head_euler_gbs": round(head_gbs, 1), "head_euler_frac_hbm": round(head_gbs / peaks["hbm_gbs"], 4),
         "gpu_launches": launches * args.steps,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,
@@ -409,7 +439,7 @@ def run_e4m3(args, w):
     stream = torch.cuda.current_stream(dev)
     calls = ["h3_embed_pack", "h3_adaln_norm_modulate_e4m3", "h3_qkv_qknorm_mrope_e4m3", "h3_attention",
              "h3_quantize_rows_e4m3", "h3_gated_residual_e4m3", "h3_adaln_norm_modulate_e4m3#2",
-             "h3_ffn_swiglu_e4m3", "h3_head_unpack", "h3_euler_step"]
+             "h3_ffn_swiglu_e4m3", "h3_head_euler"]
 
     # --qk-e4m3: q, k cross to attention as e4m3 codes (H3_QK_E4M3)
     qk_flags = h3.H3_QK_NORM_ROPE_IN_QKV | (h3.H3_QK_E4M3 if args.qk_e4m3 else 0)
@@ -434,8 +464,7 @@ def run_e4m3(args, w):
         mark(7, 0)
         h3.h3_ffn_swiglu_e4m3(d, r, st.x, st.xq, st.xs, W8["Wgu"], W8["Wgu_s"], W8["Wd"], W8["Wd_s"], mod, st.ws8)
         mark(7, 1)
-        mark(8, 0); st.head(); mark(8, 1)
-        mark(9, 0); st.euler(lat_v, lat_a, (sv[s], sv[s + 1]), (sa[s], sa[s + 1])); mark(9, 1)
+        mark(8, 0); st.head_euler(lat_v, lat_a, (sv[s], sv[s + 1]), (sa[s], sa[s + 1])); mark(8, 1)
 
     for i in range(args.warmup):
         step(i)
@@ -556,15 +585,104 @@ def run_sampler(args, w):
             "gpu_launches": smp.launches_per_step() * args.steps, "clocks": clocks}
 
 
+def run_sp(args, w):
+    """Sequence parallelism (Ulysses, "MiniMax-H3 paper reading" §7.2): one
+    packed sequence split over the N ranks of the job, one process per GPU,
+    the exchange buffers opened through CUDA IPC and the two re-shardings
+    fused into the QKV and attention epilogues (peer stores).  One timed unit
+    is one block over the whole sequence (the ranks' shards together); the
+    total work is fixed as N grows: strong scaling.  Embed, head and Euler are
+    token-local and not part of this line."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from omni_modal_diffusion_b200 import h3
+    from omni_modal_diffusion_b200.pipeline import H3BlockStep
+    from omni_modal_diffusion_b200.sp_runner import SPProcessRank
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if not (dist.is_available() and dist.is_initialized()):
+        if "MASTER_ADDR" not in os.environ:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29533")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + w.index)            # the same weights and inputs on every rank
+
+    def randn(*shape, std=1.0, dtype=torch.bfloat16):
+        return (torch.randn(*shape, generator=g, device=dev, dtype=torch.float32) * std).to(dtype)
+
+    W = {"W_text": randn(w.D, w.D_text, std=0.02), "W_vid": randn(w.D, 4 * w.C_lat, std=0.02),
+         "W_aud": randn(w.D, w.C_audio, std=0.02), "Wqkv": randn(3 * w.I, w.D, std=0.02),
+         "qn_w": (1 + 0.1 * torch.randn(128, generator=g, device=dev)).to(torch.bfloat16),
+         "kn_w": (1 + 0.1 * torch.randn(128, generator=g, device=dev)).to(torch.bfloat16),
+         "Wo": randn(w.D, w.I, std=0.02), "Wgu": randn(2 * w.F, w.D, std=0.02), "Wd": randn(w.D, w.F, std=0.02),
+         "W_vhead": randn(4 * w.C_lat, w.D, std=0.02), "W_ahead": randn(w.C_audio, w.D, std=0.02)}
+    st = H3BlockStep(w, device=dev, weights=W)
+    st.embed(randn(w.n_text, w.D_text), randn(w.T_lat, w.H_lat, w.W_lat, w.C_lat),
+             randn(w.audio_channels, w.n_audio, w.C_audio))
+    mod = randn(3, 6, w.D, std=0.1, dtype=torch.float32)
+    L = st.ranges.L
+    me = SPProcessRank(w, st.dims, st.ranges, dev)
+    r = me.rank
+    r.x.zero_()
+    r.pos.zero_()
+    lo, hi = r.rows.start, min(r.rows.stop, st.ranges.L_pad)
+    x0 = torch.zeros_like(r.x)
+    x0[: hi - lo].copy_(st.x[lo:hi])
+    r.pos[: hi - lo].copy_(st.pos[lo:hi])
+    del st                                    # only the shard stays resident
+    stream = torch.cuda.current_stream(dev)
+    me.barrier()
+    for _ in range(args.warmup):
+        r.x.copy_(x0)
+        me.block_forward(mod, W)
+    me.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        me.block_forward(mod, W)
+    t1.record(stream)
+    me.barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    status = h3.h3_device_status()
+    (ms,) = max_over_ranks([ms], device=dev)
+    me.close()
+    dist.destroy_process_group()
+    if status != 0:
+        raise RuntimeError(f"device-side wait gave up (code {status})")
+    if rank != 0:
+        return None
+    fl = block_flops(w, L)
+    return {"metric": "packed tokens/s per Omni block, sequence-parallel (Ulysses) over the job's GPUs",
+            "value": round(L / (ms / 1e3), 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/text, N(0,0.02) weights)",
+            "config": {"workload": w.name, "packed_tokens": L, "parallelism": f"ulysses sp{world}",
+                       "L_shard": me.layout.L_shard, "heads_per_rank": me.layout.heads},
+            "tflops": round(fl / (ms / 1e3) / 1e12, 1),
+            "gpu_launches": 7 * args.steps,   # LN, QKV, attention, out-projection, LN, FFN gate/up + down
+            "barriers_per_block": 2}
+
+
 def run_only(args, w):
     """One C-ABI call on the workload's shapes, nothing else resident but its
     operands (for ncu captures of a single kernel)."""
+    import dataclasses
     import torch
     from omni_modal_diffusion_b200 import h3
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev)
     g.manual_seed(4321)
     rnd = lambda *s, std=1.0, dt=torch.bfloat16: (torch.randn(*s, generator=g, device=dev) * std).to(dt)
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads)
     d = h3.make_dims(w.D, w.H, w.F, rope=w.rope_split)
     r = h3.h3_make_ranges(w.n_text, w.audio_channels * w.n_audio, w.T_lat * (w.H_lat // 2) * (w.W_lat // 2))
     Lp = r.L_pad
@@ -610,7 +728,12 @@ def run_only(args, w):
     b.record()
     torch.cuda.synchronize()
     assert h3.h3_device_status() == 0
-    print(f"{args.only} on {w.name}: {a.elapsed_time(b) / args.steps:.4f} ms per call", flush=True)
+    ms = a.elapsed_time(b) / args.steps
+    extra = ""
+    if args.only == "attention":
+        L = r.L
+        extra = f", {4.0 * L * L * w.I / (ms / 1e3) / 1e12:.1f} TFLOP/s"
+    print(f"{args.only} on {w.name} (H={w.H}): {ms:.4f} ms per call{extra}", flush=True)
 
 
 def block_flops(w, L):
@@ -618,26 +741,43 @@ def block_flops(w, L):
     return 2.0 * L * (w.D * 3 * w.I + w.I * w.D + 2 * w.D * w.F + w.F * w.D) + 4.0 * L * L * w.I
 
 
-def cpu_baseline(w, frames=2):
+_SAMPLE_CACHE = {}
+
+
+def _oracle_sample_inputs(w, frames):
+    """Seeded inputs of the cut workload and its packing, drawn once per
+    process (drawing the full-width weights takes longer than the sample)."""
+    key = (w.name, frames)
+    if key not in _SAMPLE_CACHE:
+        import dataclasses
+        from oracle import h3_oracle as O
+        from omni_modal_diffusion_b200 import synthetic as S
+        ws = dataclasses.replace(w, T_lat=min(frames, w.T_lat))
+        inp = S.make_inputs(ws)
+        t_g, i_g, j_g = O.token_grid(ws.T_lat, ws.H_lat, ws.W_lat)
+        r = O.pack_ranges(ws.n_text, ws.audio_channels * ws.n_audio, t_g * i_g * j_g)
+        pos = O.positions(r, t_g, i_g, j_g, ws.audio_channels, ws.n_audio)
+        _SAMPLE_CACHE[key] = (ws, inp, r, pos)
+    return _SAMPLE_CACHE[key]
+
+
+def cpu_baseline(w, frames=None):
     """The float64 oracle on the host cores, on a bounded sample of the same
     workload: the whole block (packing, projections, LN+modulate, QKV,
     RMSNorm, RoPE, attention, gated out-projection, SwiGLU FFN) on the same
-    text and audio with the video cut to `frames` latent frames, timed in
-    full, then scaled to the workload's length by the block's algorithmic
-    FLOPs (the oracle is matmul-bound)."""
-    import dataclasses
+    text and audio with the video cut to `frames` latent frames (2, or 1 for
+    the 15 s workload, whose 1,200 audio and 1,344 video tokens per frame
+    already make a ~6 s sample), timed in full, then scaled to the workload's
+    length by the block's algorithmic FLOPs (the oracle is matmul-bound)."""
+    if frames is None:
+        frames = 1 if w.T_lat > 60 else 2
     from oracle import h3_oracle as O
-    from omni_modal_diffusion_b200 import synthetic as S
     try:
         import threadpoolctl
         threads = max(info.get("num_threads", 0) for info in threadpoolctl.threadpool_info()) or os.cpu_count()
     except Exception:  # pragma: no cover
         threads = os.cpu_count()
-    ws = dataclasses.replace(w, T_lat=min(frames, w.T_lat))
-    inp = S.make_inputs(ws)
-    t_g, i_g, j_g = O.token_grid(ws.T_lat, ws.H_lat, ws.W_lat)
-    r = O.pack_ranges(ws.n_text, ws.audio_channels * ws.n_audio, t_g * i_g * j_g)
-    pos = O.positions(r, t_g, i_g, j_g, ws.audio_channels, ws.n_audio)
+    ws, inp, r, pos = _oracle_sample_inputs(w, frames)
     t0 = time.perf_counter()
     x = O.embed(inp["text"], inp["video"], inp["audio"], inp["W_text"], inp["W_vid"], inp["W_aud"], r)
     O.block_forward(x, inp["mod"], r, pos, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"], inp["Wgu"],
@@ -650,7 +790,7 @@ def cpu_baseline(w, frames=2):
             "sample": f"float64 oracle block on {w.name} cut to {ws.T_lat} latent frames ({Ls} packed tokens, "
                       f"{t_s:.1f} s measured), scaled to {L} tokens by algorithmic FLOPs "
                       f"({block_flops(w, L) / block_flops(w, Ls):.2f}x)",
-            "seconds_per_block_extrapolated": round(t_full, 2)}
+            "seconds_per_block_extrapolated": round(t_full, 2), "sample_seconds": round(t_s, 3)}
 
 
 def run_reference(args, w):
@@ -661,12 +801,10 @@ def run_reference(args, w):
     vals, secs = [], []
     base = None
     for i in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        cb = cpu_baseline(w)
-        dt = time.perf_counter() - t0
+        cb = cpu_baseline(w)   # times the oracle block alone (inputs drawn once, untimed)
         if i >= args.warmup:
             vals.append(cb["value"])
-            secs.append(dt)
+            secs.append(cb["sample_seconds"])
             base = cb
     value = statistics.mean(vals)
     return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -686,31 +824,40 @@ def main():
     ap.add_argument("--sampler", action="store_true",
                     help="time the layered flow sampler (denoise steps/s) instead of the single-block step")
     ap.add_argument("--layers", type=int, default=50)
+    ap.add_argument("--sp", action="store_true",
+                    help="sequence parallelism: one sequence split over the job's ranks (a separate line)")
     ap.add_argument("--e4m3", action="store_true",
                     help="the block step with its four GEMMs in e4m3 (a separate line; one GPU)")
     ap.add_argument("--qk-e4m3", action="store_true",
                     help="with --e4m3: q and k cross to attention as e4m3 codes (Q K^T on e4m3 MMAs)")
     ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln", "euler"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
+    ap.add_argument("--heads", type=int, default=None, help="with --only: this many heads instead of the workload's")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=None, help=f"default {DEFAULT_WORKLOAD}; sampler: 768x1344_5s")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    from omni_modal_diffusion_b200 import synthetic as S
+    w = S.WORKLOADS[args.workload or ("768x1344_5s" if args.sampler else DEFAULT_WORKLOAD)]
+    long_seq = w.T_lat * (w.H_lat // 2) * (w.W_lat // 2) > 60000  # ~0.5 s per block step
     if args.steps is None:
-        args.steps = 8 if args.sampler else 100
+        args.steps = 8 if args.sampler else (20 if long_seq else 100)
     if args.warmup is None:
-        args.warmup = 3 if args.sampler else 10
+        args.warmup = 3 if args.sampler else (5 if long_seq else 10)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference" and args.warmup > 1:
         args.warmup = 1            # each oracle step is a ~10-30 s CPU sample
-    from omni_modal_diffusion_b200 import synthetic as S
-    w = S.WORKLOADS[args.workload or ("768x1344_5s" if args.sampler else DEFAULT_WORKLOAD)]
     if args.only:
         run_only(args, w)
         return
     if args.sampler:
         print(json.dumps(run_sampler(args, w)), flush=True)
+        return
+    if args.sp:
+        out = run_sp(args, w)
+        if out is not None:
+            print(json.dumps(out), flush=True)
         return
     if args.e4m3:
         print(json.dumps(run_e4m3(args, w)), flush=True)
