@@ -103,8 +103,12 @@ constexpr float P_HALF_SUM_LIMIT = 65536.0f;
 #ifndef H3_ATTN_MMA_SPIN
 #define H3_ATTN_MMA_SPIN 0
 #endif
-#if H3_ATTN_MMA_SPIN
+#if H3_ATTN_MMA_SPIN == 1
 #define MMA_WAIT_WARP mbar_wait_spin_warp
+#elif H3_ATTN_MMA_SPIN == 2
+#define MMA_WAIT_WARP mbar_wait_spin_lane0
+#elif H3_ATTN_MMA_SPIN == 3
+#define MMA_WAIT_WARP mbar_wait_lane0
 #else
 #define MMA_WAIT_WARP mbar_wait_warp
 #endif
