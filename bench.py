@@ -97,7 +97,8 @@ TRAFFIC = {
     ("768sq_2s", "gemm_tc_kernel"): 1.539e9,
     # the same four launches with e4m3 operands (2.679 GB / 4)
     ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.670e9,
-    # one attention launch
+    # one attention launch of the general kernel (captured before the split
+    # kernel became the block's attention; kept for that kernel only)
     ("768sq_2s", "attention_tc_kernel"): 0.4379e9,
 }
 
@@ -236,7 +237,7 @@ def run_ours(args, w):
         mark(2, 0)
         h3.h3_qkv_qknorm_mrope(d, r, st.xm, st.W["Wqkv"], st.W["qn_w"], st.W["kn_w"], st.pos, st.q, st.k, st.v)
         mark(2, 1)
-        mark(3, 0); h3.h3_attention(d, r, st.q, st.k, st.v, st.o); mark(3, 1)
+        mark(3, 0); h3.h3_attention(d, r, st.q, st.k, st.v, st.o, qn_w=st.W["qn_w"], kn_w=st.W["kn_w"]); mark(3, 1)
         mark(4, 0); h3.h3_gated_residual(d, r, st.x, st.o, st.W["Wo"], mod, h3.H3_MSA); mark(4, 1)
         mark(5, 0); h3.h3_adaln_norm_modulate(d, r, st.x, mod, h3.H3_MLP, st.xm); mark(5, 1)
         mark(6, 0); h3.h3_ffn_swiglu(d, r, st.x, st.xm, st.W["Wgu"], st.W["Wd"], mod, st.ws); mark(6, 1)
@@ -351,20 +352,26 @@ def run_ours(args, w):
     # Kernels: the tcgen05 GEMM (gemm_tc2_kernel, CTA pairs, for QKV and the
     # out-projection; gemm_tc_kernel for the FFN's gate/up and down) runs the
     # block's four GEMM launches (the embed/head launches add < 0.4% of its
-    # FLOPs and are not timed separately); attention_tc_kernel is one launch.
+    # FLOPs and are not timed separately).  h3_attention with the norm
+    # weights is attention_split_kernel plus the general kernel's fixup launch
+    # (whose CTAs return at once unless the split kernel left them work).
     gemm_calls = ("h3_qkv_qknorm_mrope", "h3_gated_residual", "h3_ffn_swiglu")
     gemm_ms = sum(per_call[c] for c in gemm_calls)
     gemm_tf = sum(fl[c] for c in gemm_calls) / (gemm_ms / 1e3) / 1e12
     attn_tf = tensor_calls["h3_attention"]
     kernels = {"gemm_tc_kernel": kernel_entry(gemm_ms, 4, gemm_tf, peak_tf, peaks,
                                               TRAFFIC.get((w.name, "gemm_tc_kernel"))),
-               "attention_tc_kernel": kernel_entry(per_call["h3_attention"], 1, attn_tf, peak_tf, peaks,
-                                                   TRAFFIC.get((w.name, "attention_tc_kernel")))}
+               "attention_split_kernel": kernel_entry(per_call["h3_attention"], 1, attn_tf, peak_tf, peaks,
+                                                      TRAFFIC.get((w.name, "attention_split_kernel")))}
     dominant = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     block_flops = sum(fl.values())
     block_ms = sum(per_call[c] for c in ("h3_adaln_norm_modulate", "h3_qkv_qknorm_mrope", "h3_attention",
                                          "h3_gated_residual", "h3_adaln_norm_modulate#2", "h3_ffn_swiglu"))
-    ln_gbs = by["h3_adaln_norm_modulate"] / (per_call["h3_adaln_norm_modulate"] / 1e3) / 1e9
+    # the two LN + modulate launches of the block (attention and FFN branch)
+    ln_each = [by["h3_adaln_norm_modulate"] / (per_call[c] / 1e3) / 1e9
+               for c in ("h3_adaln_norm_modulate", "h3_adaln_norm_modulate#2")]
+    ln_gbs = 2 * by["h3_adaln_norm_modulate"] / ((per_call["h3_adaln_norm_modulate"]
+                                                  + per_call["h3_adaln_norm_modulate#2"]) / 1e3) / 1e9
     head_gbs = by["h3_head_euler"] / (per_call["h3_head_euler"] / 1e3) / 1e9
     launches = st.launches_per_step()
     out = {
@@ -392,6 +399,7 @@ def run_ours(args, w):
         "per_call_ms": {c: round(v, 4) for c, v in per_call.items()},
         "per_call_tflops": {c: round(v, 1) for c, v in tensor_calls.items()},
         "ln_modulate_gbs": round(ln_gbs, 1), "ln_modulate_frac_hbm": round(ln_gbs / peaks["hbm_gbs"], 4),
+        "ln_modulate_per_launch_gbs": [round(v, 1) for v in ln_each],
         "head_euler_gbs": round(head_gbs, 1), "head_euler_frac_hbm": round(head_gbs / peaks["hbm_gbs"], 4),
         "gpu_launches": launches * args.steps,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -513,13 +521,14 @@ def run_e4m3(args, w):
         "kernels": {"gemm_tc_kernel<e4m3>": {"ms_per_step": round(gemm_ms, 4), "tflops": round(gemm_tf, 1),
                                              "frac": round(gemm_tf / peak_f8, 4), "launches_per_step": 4,
                                              "traffic_per_launch": TRAFFIC.get((w.name, "gemm_tc_kernel<e4m3>"))},
-                    "attention_tc_kernel": {"ms_per_step": round(per_call["h3_attention"], 4),
+                    ("attention_tc_kernel<e4m3 QK>" if args.qk_e4m3 else "attention_split_kernel"): {
+                                            "ms_per_step": round(per_call["h3_attention"], 4),
                                             "tflops": round(fl["h3_attention"] / (per_call["h3_attention"] / 1e3)
                                                             / 1e12, 1)}},
         "block": {"ms": round(block_ms, 4),
                   "tflops": round(sum(fl.values()) / (block_ms / 1e3) / 1e12, 1)},
         "per_call_ms": {c: round(v, 4) for c, v in per_call.items()},
-        "gpu_launches": st.launches_per_step(e4m3=True) * args.steps,
+        "gpu_launches": st.launches_per_step(e4m3=True, qk_e4m3=args.qk_e4m3) * args.steps,
         "clocks": clocks,
     }
 
@@ -667,7 +676,7 @@ def run_sp(args, w):
             "config": {"workload": w.name, "packed_tokens": L, "parallelism": f"ulysses sp{world}",
                        "L_shard": me.layout.L_shard, "heads_per_rank": me.layout.heads},
             "tflops": round(fl / (ms / 1e3) / 1e12, 1),
-            "gpu_launches": 7 * args.steps,   # LN, QKV, attention, out-projection, LN, FFN gate/up + down
+            "gpu_launches": 8 * args.steps,   # LN, QKV, attention (split + fixup), out-projection, LN, FFN x2
             "barriers_per_block": 2}
 
 
@@ -687,10 +696,23 @@ def run_only(args, w):
     r = h3.h3_make_ranges(w.n_text, w.audio_channels * w.n_audio, w.T_lat * (w.H_lat // 2) * (w.W_lat // 2))
     Lp = r.L_pad
     mod = rnd(3, 6, w.D, std=0.1, dt=torch.float32)
-    if args.only == "attention":
+    if args.only in ("attention", "attention_raw"):
+        # q, k rows as the QKV call leaves them: RMS-normalised and scaled by
+        # the norm weights (attention then runs its split-softmax kernel);
+        # attention_raw: unnormalised N(0, 1) rows, no norm weights (the
+        # general kernel alone)
         q, k, v = (rnd(w.H, Lp, 128) for _ in range(3))
+        qn, kn = rnd(128, std=0.1) + 1, rnd(128, std=0.1) + 1
+        if args.only == "attention":
+            def rms(x, wt):
+                xf = x.float()
+                return (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + 1e-6) * wt.float()).to(torch.bfloat16)
+            q, k = rms(q, qn), rms(k, kn)
         o = torch.empty(Lp, w.I, dtype=torch.bfloat16, device=dev)
-        fn = lambda: h3.h3_attention(d, r, q, k, v, o)
+        if args.only == "attention":
+            fn = lambda: h3.h3_attention(d, r, q, k, v, o, qn_w=qn, kn_w=kn)
+        else:
+            fn = lambda: h3.h3_attention(d, r, q, k, v, o)
     elif args.only == "qkv":
         xm = rnd(Lp, w.D)
         Wqkv = rnd(3 * w.I, w.D, std=0.02)
@@ -730,7 +752,7 @@ def run_only(args, w):
     assert h3.h3_device_status() == 0
     ms = a.elapsed_time(b) / args.steps
     extra = ""
-    if args.only == "attention":
+    if args.only.startswith("attention"):
         L = r.L
         extra = f", {4.0 * L * L * w.I / (ms / 1e3) / 1e12:.1f} TFLOP/s"
     print(f"{args.only} on {w.name} (H={w.H}): {ms:.4f} ms per call{extra}", flush=True)
@@ -830,7 +852,7 @@ def main():
                     help="the block step with its four GEMMs in e4m3 (a separate line; one GPU)")
     ap.add_argument("--qk-e4m3", action="store_true",
                     help="with --e4m3: q and k cross to attention as e4m3 codes (Q K^T on e4m3 MMAs)")
-    ap.add_argument("--only", default=None, choices=["attention", "qkv", "out", "ffn", "ln", "euler"],
+    ap.add_argument("--only", default=None, choices=["attention", "attention_raw", "qkv", "out", "ffn", "ln", "euler"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--heads", type=int, default=None, help="with --only: this many heads instead of the workload's")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -150,7 +150,15 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
 /* A6.  o = softmax(q k^T / sqrt(128)) v per head over all L valid tokens,
  * non-causal; keys >= L are masked ([shouss] §5).  q, k, v: head-major
  * [H][L_pad][128] bf16 as written by h3_qkv_qknorm_mrope (flags must carry
- * H3_QK_NORM_ROPE_IN_QKV; qn_w, kn_w and pos are then unused and may be NULL).
+ * H3_QK_NORM_ROPE_IN_QKV; pos is unused and may be NULL).
+ *   qn_w, kn_w: the norm weights q and k were normalised with, or both NULL.
+ *     Given (bf16 q, k), the softmax needs no running maximum: every score
+ *     lies within sqrt(128) max|qn_w| max|kn_w| of 0, so the exponentials are
+ *     taken against that bound, each row's over two warps.  A CTA whose
+ *     scores break the bound (q, k not normalised as stated) or whose bound
+ *     is too wide for fp32 (scores past +-60 in log2 units) is recomputed by
+ *     the general kernel in a second launch: the result is the same either
+ *     way.  NULL: the general kernel (moving softmax reference) alone.
  * With flags & H3_QK_E4M3, q and k are the e4m3 codes written by
  * h3_qkv_qknorm_mrope_e4m3 with that flag (one byte per element) and qn_w,
  * kn_w are required: the code scales follow from them.
@@ -480,9 +488,11 @@ int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3
  * peers->q/k/v[rank], filled by every rank's h3_qkv_qknorm_mrope_sp), with
  * output row R (global) written to peers->o[R / L_shard], row R % L_shard,
  * columns of head (rank H/N + h): attention and the second all-to-all in
- * one kernel.  Rows >= L are written as 0. */
-int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers, int flags,
-                    void* stream);
+ * one kernel.  Rows >= L are written as 0.  qn_w, kn_w: as for
+ * h3_attention (the norm weights q and k were normalised with, selecting
+ * the split-softmax kernel, or both NULL). */
+int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers,
+                    const h3_bf16* qn_w, const h3_bf16* kn_w, int flags, void* stream);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,418 @@
+// Non-causal flash attention with each query row's exponentials split over
+// two warps ("MiniMax-H3: native joint audio-video generation"
+// (note.shouss.top) §5: full attention over the packed sequence).
+//
+// Same work split as attention_tc_kernel (one CTA per pair of 128-query
+// tiles of one head, S and O in TMEM, P written back over S as bf16, the MMA
+// warp issuing P V and the next S of one tile while the other tile's softmax
+// runs), but each (query tile, TMEM lane quarter) has two softmax warps, one
+// per 64-key half of the key tile.  The two warps of a quarter share one
+// sub-partition and its MUFU unit: while one waits on its exponentials or on
+// TMEM the other issues, so a tile's softmax phase approaches the MUFU time
+// of its 16,384 exponentials instead of one warp's latency chain.
+//
+//   Warp 0       TMA producer (Q tiles once, K/V through 2-stage rings)
+//   Warp 1       TMEM owner and MMA issuer
+//   Warps 2-17   softmax: tile t = (w - 2) / 8, key half hf = ((w - 2) / 4) % 2,
+//                lane quarter w % 4 (the quarter a warp may access in TMEM)
+//
+// The two halves of a row cannot move a softmax reference independently (O
+// accumulates both halves' P V against one reference), and agreeing on it
+// every key tile would put a handshake on each tile's critical path.  So
+// this kernel takes no running maximum at all: q and k as the QKV call
+// writes them are RMS-normalised rows scaled by the norm weights qn_w, kn_w,
+// so ||q|| <= sqrt(128) max|qn_w|, ||k|| <= sqrt(128) max|kn_w| (bf16
+// rounding adds at most 2^-8 to the product), and every score in log2 units
+// is within B = 16.32 max|qn_w| max|kn_w| (1.01 margin) of 0.  Each p is taken
+// as 2^(x - B) <= 1: no overflow, and with B <= 60 no p falls below 2^-120,
+// so nothing flushes.  A CTA whose scores break the bound (a key-half sum
+// above 2^32: q, k not normalised as stated) or whose norm weights give
+// B > 60 leaves a NaN sentinel in its first output element instead of its
+// rows, and a second launch of attention_tc_kernel recomputes exactly those
+// CTAs with its moving reference.
+#include "h3_internal.cuh"
+#include "ptx.cuh"
+
+namespace h3 {
+
+namespace attn_split {
+using attn_detail::AttnOut;
+using attn_detail::HALF_BYTES;
+using attn_detail::TILE;
+using attn_detail::TILE_BYTES;
+using attn_detail::TMEM_COLS;
+
+constexpr int NUM_THREADS = 18 * 32;
+// Order of the MMA warp's waits and stage releases: 1 puts every wait and
+// commit that is not on a P -> P V path where the warp waits for P anyway
+// (V(j) before tile 0's first P half, K(j + 1) after tile 0's first P V half,
+// the releases of K(j) and V(j - 1) after that half; needs a third V stage);
+// 0 waits for V and K right before the MMAs that read them and releases
+// each stage after its last MMA.
+#ifndef H3_ATTN_SPLIT_ORDER
+#define H3_ATTN_SPLIT_ORDER 0
+#endif
+constexpr int SVS = H3_ATTN_SPLIT_ORDER ? 3 : 2;  // V stages
+constexpr int SQ = 0;                       // 2 query tiles
+constexpr int SK = SQ + 2 * TILE_BYTES;     // 2 stages
+constexpr int SV = SK + 2 * TILE_BYTES;     // SVS stages
+constexpr int SBAR = SV + SVS * TILE_BYTES;
+constexpr int BYTES = SBAR + 256 + 1024;
+// [2 tiles][2 halves][128 rows] row sums, written after a warp's key loop:
+// over the K stage that held K(nkv - 2), whose last S MMA completed before
+// any tile's last S (the other stage may still feed the other tile's last S)
+constexpr int SSUM = SK;
+static_assert(BYTES <= 232448, "shared memory per CTA");
+constexpr float B_MAX = 60.0f;              // largest bound whose p stay >= 2^-120
+constexpr float HALF_SUM_LIMIT = 4294967296.0f;  // 2^32: a key half above it breaks the bound
+
+// 32 lanes x 16 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// Where the first output element of the CTA's first query tile lives.
+__device__ __forceinline__ bf16* sentinel_ptr(const AttnOut& out, int grow, int h) {
+  const int owner = grow / out.L_shard;
+  return out.shard[owner] + (long)(grow - owner * out.L_shard) * out.ld + (out.head0 + h) * 128;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attention_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnOut out, int H,
+                           int L, int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = smem + SQ;
+  uint8_t* sK = smem + SK;
+  uint8_t* sV = smem + SV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SBAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [SVS]
+  uint64_t* v_empty = bars + 8;   // [SVS]
+  uint64_t* s_full = bars + 11;   // [2] per query tile
+  uint64_t* o_final = bars + 13;  // [2] per query tile
+  uint64_t* p_full = bars + 15;   // [2 tiles][2 halves]: 4 warp arrivals each
+  uint64_t* drain = bars + 19;
+  uint64_t* sums_done = bars + 20;  // [2] every softmax warp has written its row sums / its low-side verdict
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  float* bound = reinterpret_cast<float*>(bars + 23);
+  int* cta_bad = reinterpret_cast<int*>(bars + 24);
+  float* lsum = reinterpret_cast<float*>(smem + SSUM + (((L + TILE - 1) / TILE) & 1) * TILE_BYTES);  // [t][hf][row]
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_qt = L_pad / TILE;
+  const int qt0 = blockIdx.x * 2;
+  const bool two = qt0 + 1 < n_qt;
+  const int nt = two ? 2 : 1;
+  const int qt1 = two ? qt0 + 1 : qt0;
+  const int h = blockIdx.y;
+  const int nkv = (L + TILE - 1) / TILE;
+  const int row0 = h * L_pad;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&o_final[s], 1);
+      mbar_init(&p_full[2 * s], 4);
+      mbar_init(&p_full[2 * s + 1], 4);
+    }
+    for (int s = 0; s < SVS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(drain, 1);
+    mbar_init(&sums_done[0], 8 * nt);
+    mbar_init(&sums_done[1], 8 * nt);
+    *cta_bad = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    float mq = 0.f, mk = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      mq = fmaxf(mq, fabsf(__bfloat162float(qn_w[lane * 4 + i])));
+      mk = fmaxf(mk, fabsf(__bfloat162float(kn_w[lane * 4 + i])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
+      mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+    }
+    // 128 mq mk (1 + 2^-9)^2 log2(e) / sqrt(128), with a 1% margin
+    if (lane == 0) *bound = 16.3219f * 1.01f * mq * mk;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float B = *bound;
+  const bool fast = B <= B_MAX;  // uniform across the CTA
+
+  if (!fast) {
+    // the bound is too wide for p to stay normal: leave the CTA to the
+    // recomputing launch
+    if (threadIdx.x == 0) *sentinel_ptr(out, qt0 * TILE, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
+  } else if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, nt * TILE_BYTES);
+      for (int t = 0; t < nt; ++t) {
+        const int qrow = row0 + (t == 0 ? qt0 : qt1) * TILE;
+        tma_load_2d(sQ + t * TILE_BYTES, &tmQ, q_full, 0, qrow);
+        tma_load_2d(sQ + t * TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, qrow);
+      }
+      long long k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) break;
+        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
+        tma_load_2d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, row0 + j * TILE);
+        tma_load_2d(sK + st * TILE_BYTES + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
+        ++k_issued;
+        const int sv = j % SVS;
+        if (!mbar_wait(&v_empty[sv], ((j / SVS) & 1) ^ 1)) break;
+        mbar_arrive_expect_tx(&v_full[sv], TILE_BYTES);
+        tma_load_2d(sV + sv * TILE_BYTES, &tmV, &v_full[sv], 0, row0 + j * TILE);
+        tma_load_2d(sV + sv * TILE_BYTES + HALF_BYTES, &tmV, &v_full[sv], 64, row0 + j * TILE);
+        ++v_issued;
+      }
+      mbar_wait(q_full, 0);
+      drain_loads(k_full, 2, k_issued);
+      drain_loads(v_full, SVS, v_issued);
+    }
+  } else if (warp == 1) {
+    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);  // V is MN-major
+    const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t v_desc = sdesc_sw128(smem_u32(sV), HALF_BYTES, 1024);
+    auto issue_s = [&](int t, int j) {
+      const uint64_t qd = q_desc + (uint64_t)((t * TILE_BYTES) >> 4);
+      const uint64_t kd = k_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+        umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[t]);
+    };
+    // O_t += P_t V_j for keys [64 hf, 64 hf + 64): that half's P sits in
+    // TMEM columns [64 hf, 64 hf + 32) of the tile's S region
+    auto issue_pv_half = [&](int t, int j, int hf) {
+      const uint64_t vd = v_desc + (uint64_t)(((j % SVS) * TILE_BYTES) >> 4);
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = hf * 4 + k4;
+        umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + hf * 64 + k4 * 8,
+                         vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j | kk) != 0 ? 1u : 0u);
+      }
+    };
+    bool ok = mbar_wait_warp(q_full, 0) && mbar_wait_warp(&k_full[0], 0);
+#if H3_ATTN_SPLIT_ORDER
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      if (two) issue_s(1, 0);
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
+      const bool more = j + 1 < nkv;
+      if (!mbar_wait_warp_fast(&v_full[j % SVS], (j / SVS) & 1)) { ok = false; break; }
+      for (int t = 0; t < nt; ++t) {
+        if (!mbar_wait_warp_fast(&p_full[2 * t], j & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv_half(t, j, 0);
+        if (t == 0) {
+          umma_commit(&k_empty[j & 1]);                     // K(j): its last S MMA was issued a step ago
+          if (j > 0) umma_commit(&v_empty[(j - 1) % SVS]);  // V(j - 1): its last P V likewise
+          if (more && !mbar_wait_warp_fast(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
+        }
+        if (!mbar_wait_warp_fast(&p_full[2 * t + 1], j & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv_half(t, j, 1);
+        if (more)
+          issue_s(t, j + 1);
+        else
+          umma_commit(&o_final[t]);
+      }
+    }
+#else
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      if (two) issue_s(1, 0);
+      umma_commit(&k_empty[0]);
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
+      const bool more = j + 1 < nkv;
+      for (int t = 0; t < nt && ok; ++t) {
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!mbar_wait_warp(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
+          if (t == 0 && hf == 0 && !mbar_wait_warp(&v_full[j % SVS], (j / SVS) & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv_half(t, j, hf);
+        }
+        if (!ok) break;
+        if (more) {
+          if (t == 0) {
+            if (!mbar_wait_warp(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_s(t, j + 1);
+          if (t == nt - 1) umma_commit(&k_empty[(j + 1) & 1]);
+        } else {
+          umma_commit(&o_final[t]);
+        }
+      }
+      umma_commit(&v_empty[j % SVS]);
+    }
+#endif
+    drain_mmas(drain);
+  } else if (((warp - 2) >> 3) < nt) {
+    const int t = (warp - 2) >> 3;         // query tile
+    const int hf = ((warp - 2) >> 2) & 1;  // key half of every key tile
+    const int qw = warp & 3;               // TMEM lane quarter
+    const int r = qw * 32 + lane;          // query row inside the tile
+    const uint32_t tS = tmem + ((uint32_t)(qw * 32) << 16) + t * 256;
+    const uint32_t tH = tS + hf * 64;      // this warp's 64 score columns; its P goes to the first 32
+    const uint32_t tO = tS + 128;
+    const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+    const uint64_t nb2 = f2_pack(-B, -B);
+    float l_part = 0.f;
+    bool bad = false;
+    bool ok = true;
+    // p = 2^(s scale_log2 - B) for 32 scores; their bf16 pairs into pk[16];
+    // returns their sum (masked keys, -inf, give 0)
+    auto exp32 = [&](const float* s, uint32_t* pk) {
+      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nb2), x0, x1);
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_pack(p0, p1));
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      float a0, a1, a2, a3;
+      f2_unpack(acc[0], a0, a1);
+      f2_unpack(acc[1], a2, a3);
+      return (a0 + a1) + (a2 + a3);
+    };
+    for (int j = 0; j < nkv; ++j) {
+      ok = mbar_wait_warp(&s_full[t], j & 1);
+      if (!ok) break;
+      tc_fence_after();
+      const int valid = L - j * TILE - hf * 64;  // this half's keys [0, valid) are real
+      float s[32];
+      uint32_t pkA[16], pkB[16];
+      tmem_ld32(tH, reinterpret_cast<uint32_t*>(s));
+      tmem_wait_ld();
+      if (valid < 32) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      float hs = exp32(s, pkA);
+      // P of keys [0, 32) of the half over its own first 16 score columns
+      tmem_st16(tH, pkA);
+      tmem_ld32(tH + 32, reinterpret_cast<uint32_t*>(s));
+      tmem_wait_ld();
+      if (valid < 64) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (c + 32 >= valid) s[c] = -INFINITY;
+      }
+      hs += exp32(s, pkB);
+      // P of keys [32, 64) of the half over score columns [16, 32), already read
+      tmem_st16(tH + 16, pkB);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[2 * t + hf]);
+      bad |= !(hs <= HALF_SUM_LIMIT);
+      l_part += hs;
+    }
+    // The CTA's verdict on the bound, in two rounds so that every warp
+    // decides before any writes: (1) a key half summed past 2^32 (a score
+    // far above the bound) and the half sums; (2) a row whose whole sum fell
+    // below 2^-110 (every score far below the bound: p would flush)
+    const int qt = t == 0 ? qt0 : qt1;
+    const int grow = qt * TILE + r;
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(cta_bad, 1);
+    lsum[(t * 2 + hf) * 128 + r] = l_part;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sums_done[0]);
+    ok = mbar_wait_warp(&sums_done[0], 0) && ok;
+    const float l = lsum[(t * 2) * 128 + r] + lsum[(t * 2 + 1) * 128 + r];
+    if (__any_sync(0xffffffffu, grow < L && !(l >= 7.7e-34f)) && lane == 0) atomicOr(cta_bad, 1);  // 2^-110
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sums_done[1]);
+    if (ok) ok = mbar_wait_warp(&sums_done[1], 0) && mbar_wait_warp(&o_final[t], 0);
+    if (ok) {
+      tc_fence_after();
+      const bool redo = *reinterpret_cast<volatile int*>(cta_bad) != 0;
+      if (redo) {
+        if (t == 0 && hf == 0 && r == 0) *sentinel_ptr(out, grow, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
+      } else {
+        const float inv = (grow < L) ? 1.0f / l : 0.0f;
+        bf16* dst = sentinel_ptr(out, grow, h);
+        // this warp writes O columns [64 hf, 64 hf + 64) of its row
+#pragma unroll 1
+        for (int c = 2 * hf; c < 2 * hf + 2; ++c) {
+          float o[32];
+          tmem_ld32(tO + c * 32, reinterpret_cast<uint32_t*>(o));
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 32; d += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(o[d] * inv, o[d + 1] * inv);
+            w.y = pack_bf16x2(o[d + 2] * inv, o[d + 3] * inv);
+            w.z = pack_bf16x2(o[d + 4] * inv, o[d + 5] * inv);
+            w.w = pack_bf16x2(o[d + 6] * inv, o[d + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + c * 32 + d) = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace attn_split
+
+cudaError_t launch_attention_split(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                   const attn_detail::AttnOut& out, dim3 grid, int H, int L, int L_pad,
+                                   float scale_log2, const bf16* qn_w, const bf16* kn_w, cudaStream_t stream) {
+  static unsigned long long attr_done = 0;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(attn_split::attention_split_kernel),
+                                   attn_split::BYTES, &attr_done);
+  if (e != cudaSuccess) return e;
+  attn_split::attention_split_kernel<<<grid, attn_split::NUM_THREADS, attn_split::BYTES, stream>>>(
+      tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w);
+  return cudaGetLastError();
+}
+
+}  // namespace h3

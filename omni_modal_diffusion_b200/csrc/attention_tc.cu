@@ -19,14 +19,11 @@
 //              back over S in TMEM as packed bf16 in two halves of 64 keys,
 //              each released to the PV MMA as soon as it is stored, finally
 //              O / l to global memory.
-// The two softmax warpgroups take turns: tile 1's exponentials of key tile j
-// start when tile 0's have finished, tile 0's of key tile j + 1 when tile 1's
-// of j have (an mbarrier handoff), so each phase has the MUFU units and the
-// issue slots of all four sub-partitions to itself while the tensor core runs
-// the other tile's P V and next S.  A fixed share of each row's exponentials
-// (H3_ATTN_POLY_COLS of every 16 columns) is taken on the FMA pipe instead
-// (exp2_fma2), which shortens a phase below the MUFU-only 1,024 clocks of a
-// 128 x 128 tile (16 exponentials per clock per SM).
+// Optionally (H3_ATTN_POLY_COLS of every 16 columns, default 0) part of each
+// row's exponentials are taken on the FMA pipe (exp2_fma2) instead of the
+// MUFU unit; measured slower on B200.  attention_split_kernel
+// (attention_split.cu) replaces this kernel when q and k come with their norm
+// weights; this one then recomputes only the CTAs that kernel leaves to it.
 // With an odd number of query tiles the last CTA runs tile 0 alone.
 // TMEM (512 columns): tile t owns columns [256t, 256t + 128) for S / P and
 // [256t + 128, 256t + 256) for O.
@@ -55,15 +52,9 @@ constexpr int NUM_THREADS = 320;
 constexpr int TILE = 128;
 constexpr int HALF_BYTES = TILE * 64 * 2;   // 128 rows x 64 bf16 = 16 KB
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 32 KB
-// Stages of the V ring (2 or 3).  K keeps 2: a K tile is needed one key step
-// later than the V tile loaded before it.
-#ifndef H3_ATTN_V_STAGES
-#define H3_ATTN_V_STAGES 2
-#endif
-constexpr int VS = H3_ATTN_V_STAGES;
-static_assert(VS == 2 || VS == 3, "H3_ATTN_V_STAGES: 2 or 3");
 // Q and K tiles: bf16 (32 KB, two 64-column halves) or, with QK8, e4m3 codes
 // (16 KB, one 128-byte row per token)
+constexpr int VS = 2;  // V stages
 template <bool QK8> struct Layout {
   static constexpr int QK_TILE = QK8 ? TILE * 128 : TILE_BYTES;
   static constexpr int Q = 0;                  // 2 query tiles
@@ -81,11 +72,6 @@ constexpr int TMEM_COLS = 512;
 #endif
 static_assert(H3_ATTN_POLY_COLS >= 0 && H3_ATTN_POLY_COLS <= 16 && H3_ATTN_POLY_COLS % 2 == 0,
               "H3_ATTN_POLY_COLS: an even count of 0..16");
-// The two softmax warpgroups take turns on the exponentials (1) or run
-// whenever their S is ready (0).
-#ifndef H3_ATTN_TURNS
-#define H3_ATTN_TURNS 0
-#endif
 // S is read from TMEM in two 64-key halves (1: half 1 is loaded while P of
 // half 0 is stored, and only 64 scores are live in registers at a time) or
 // whole (0).
@@ -103,12 +89,8 @@ constexpr float P_HALF_SUM_LIMIT = 65536.0f;
 #ifndef H3_ATTN_MMA_SPIN
 #define H3_ATTN_MMA_SPIN 0
 #endif
-#if H3_ATTN_MMA_SPIN == 1
+#if H3_ATTN_MMA_SPIN
 #define MMA_WAIT_WARP mbar_wait_spin_warp
-#elif H3_ATTN_MMA_SPIN == 2
-#define MMA_WAIT_WARP mbar_wait_spin_lane0
-#elif H3_ATTN_MMA_SPIN == 3
-#define MMA_WAIT_WARP mbar_wait_lane0
 #else
 #define MMA_WAIT_WARP mbar_wait_warp
 #endif
@@ -130,7 +112,15 @@ template <bool QK8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnOut out, int H, int L,
-                        int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w) {
+                        int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w, int fixup) {
+  // fixup: recompute only the CTAs that attention_split_kernel left to this
+  // kernel (a NaN sentinel, bf16 0x7FC0, in their first output element)
+  if (fixup) {
+    const int g = blockIdx.x * 2 * TILE;
+    const int owner = g / out.L_shard;
+    const bf16* first = out.shard[owner] + (long)(g - owner * out.L_shard) * out.ld + (out.head0 + blockIdx.y) * 128;
+    if (__bfloat16_as_ushort(*first) != (unsigned short)0x7FC0) return;
+  }
   using LY = Layout<QK8>;
   constexpr int QK_TILE = LY::QK_TILE;
   extern __shared__ uint8_t smem_raw[];
@@ -150,7 +140,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* p_full = bars + 15;   // [2 tiles][2 halves of the key tile]: P half in TMEM (4 warp arrivals)
   uint64_t* drain = bars + 19;    // the MMA issuer's last commit before teardown
   uint64_t* pv0_done = bars + 20; // [2] per query tile: PV on the first key half complete
-  uint64_t* turn = bars + 22;     // [2] per query tile: its exponentials of a key tile done (4 warp arrivals)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   float* qk_scale = reinterpret_cast<float*>(bars + 25);  // QK8: dequantisation of S
 
@@ -174,7 +163,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&p_full[2 * s + 1], 4);
       mbar_init(&pv0_done[s], 1);
       mbar_init(&o_final[s], 1);
-      mbar_init(&turn[s], 4);
     }
     for (int s = 0; s < VS; ++s) {
       mbar_init(&v_full[s], 1);
@@ -329,7 +317,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1));
+      ok = mbar_wait_warp(&s_full[t], j & 1);
       if (!ok) break;
       tc_fence_after();
       float s[128];
@@ -366,19 +354,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (with S in halves: the first half's max; the second half of the
       // first key tile then takes the overflow check like any later half)
       if (j == 0) m_ref = row_max(0, 32 * kFirstLoad) * sl2;
-      // wait for the other tile's exponentials (of key tile j - 1 for tile 0,
-      // of key tile j for tile 1) to finish
-      if (H3_ATTN_TURNS && two && (t == 1 || j > 0)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&turn[1 - t], (uint32_t)((j - (t == 0 ? 1 : 0)) & 1)));
-        if (!ok) break;
-      }
       const uint64_t sc2 = f2_pack(sl2, sl2);
       // p = 2^(s * sl2 - m_ref); returns this row's sum over the half.  The
       // last key tile (masked keys at -inf, which give exactly 0) takes every
       // exponential on the MUFU unit; the others take H3_ATTN_POLY_COLS of
       // every 16 on the FMA pipe.
       auto exp_half = [&](int hf, uint32_t* pk, auto poly_tag) {
-        constexpr bool kPoly = decltype(poly_tag)::value;
+        constexpr int kPolyCols = decltype(poly_tag)::value;  // of every 16 columns
         const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
         const float pa = sl2 * (1.0f / 252.0f), pb = (125.0f - m_ref) * (1.0f / 252.0f);
         uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -386,7 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < 64; c += 2) {
           const int cc = hf * 64 + c;
           uint64_t p2;
-          if (kPoly && (c & 15) < H3_ATTN_POLY_COLS) {
+          if (kPolyCols > 0 && (c & 15) < kPolyCols) {
             p2 = exp2_fma2(s[cc], s[cc + 1], pa, pb);
           } else {
             float x0, x1;
@@ -403,11 +385,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         f2_unpack(acc[1], a2, a3);
         return (a0 + a1) + (a2 + a3);
       };
+      using NoPoly = std::integral_constant<int, 0>;
       auto exp_half_sel = [&](int hf, uint32_t* pk) {
-        if constexpr (H3_ATTN_POLY_COLS > 0)
-          return valid < TILE ? exp_half(hf, pk, std::false_type{}) : exp_half(hf, pk, std::true_type{});
-        else
-          return exp_half(hf, pk, std::false_type{});
+        if (valid < TILE) return exp_half(hf, pk, NoPoly{});
+        return exp_half(hf, pk, std::integral_constant<int, H3_ATTN_POLY_COLS>{});
       };
       float hsum[2];
       // P for keys [64 hf, 64 hf + 64) goes to TMEM columns [32 hf, 32 hf + 32)
@@ -474,7 +455,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[2 * t + hf]);
       }
       if (!ok) break;
-      if (H3_ATTN_TURNS && two && lane == 0) mbar_arrive(&turn[t]);
       l_sum += hsum[0] + hsum[1];
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
@@ -519,6 +499,12 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 bool make_tmap_e4m3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
                     uint32_t box_rows);
 
+// attention_split.cu: the split-softmax kernel on q, k normalised as the QKV
+// call writes them
+cudaError_t launch_attention_split(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                   const attn_detail::AttnOut& out, dim3 grid, int H, int L, int L_pad,
+                                   float scale_log2, const bf16* qn_w, const bf16* kn_w, cudaStream_t stream);
+
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
   const bool qk8 = p.qk8 != 0;
   if (qk8 && (p.qn_w == nullptr || p.kn_w == nullptr)) return cudaErrorInvalidValue;
@@ -553,12 +539,25 @@ cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
     out.shard[0] = p.o;
   }
   dim3 grid((n_qt + 1) / 2, p.H);
-  if (qk8)
+  if (qk8) {
     attention_tc_kernel<true><<<grid, attn_detail::NUM_THREADS, Layout<true>::BYTES, stream>>>(
-        tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, p.qn_w, p.kn_w);
-  else
+        tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, p.qn_w, p.kn_w, 0);
+    return cudaGetLastError();
+  }
+#ifndef H3_ATTN_SPLIT
+#define H3_ATTN_SPLIT 1
+#endif
+  if (H3_ATTN_SPLIT && p.qn_w != nullptr && p.kn_w != nullptr) {
+    // the split-softmax kernel on normalised q, k; then this kernel on the
+    // CTAs it left (usually none: each such CTA returns at once)
+    aerr = launch_attention_split(tq, tk, tv, out, grid, p.H, p.L, p.L_pad, p.scale_log2, p.qn_w, p.kn_w, stream);
+    if (aerr != cudaSuccess) return aerr;
     attention_tc_kernel<false><<<grid, attn_detail::NUM_THREADS, Layout<false>::BYTES, stream>>>(
-        tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, nullptr, nullptr);
+        tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, nullptr, nullptr, 1);
+    return cudaGetLastError();
+  }
+  attention_tc_kernel<false><<<grid, attn_detail::NUM_THREADS, Layout<false>::BYTES, stream>>>(
+      tq, tk, tv, out, p.H, p.L, p.L_pad, p.scale_log2, nullptr, nullptr, 0);
   return cudaGetLastError();
 }
 

@@ -13,6 +13,7 @@
 #include "elementwise.cu"
 #include "gemm_tc.cu"
 #include "attention_tc.cu"
+#include "attention_split.cu"
 
 using namespace h3;
 
@@ -325,9 +326,12 @@ int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q,
     H3_REQUIRE_PTR(qn_w);
     H3_REQUIRE_PTR(kn_w);
     p.qk8 = 1;
-    p.qn_w = reinterpret_cast<const bf16*>(qn_w);
-    p.kn_w = reinterpret_cast<const bf16*>(kn_w);
+  } else if (qn_w || kn_w) {  // bf16 q, k normalised with these weights: the split-softmax kernel
+    H3_REQUIRE_PTR(qn_w);
+    H3_REQUIRE_PTR(kn_w);
   }
+  p.qn_w = reinterpret_cast<const bf16*>(qn_w);
+  p.kn_w = reinterpret_cast<const bf16*>(kn_w);
   p.q = reinterpret_cast<const bf16*>(q);
   p.k = reinterpret_cast<const bf16*>(k);
   p.v = reinterpret_cast<const bf16*>(v);

@@ -118,8 +118,8 @@ int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3
   return ok();
 }
 
-int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers, int flags,
-                    void* stream) {
+int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers,
+                    const h3_bf16* qn_w, const h3_bf16* kn_w, int flags, void* stream) {
   H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_layout(dims, layout, __func__));
@@ -133,8 +133,14 @@ int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp
     return fail(H3_ERR_NULL, "%s: this rank's q, k, v buffers are required", __func__);
   if (!aligned16(peers->q[r]) || !aligned16(peers->k[r]) || !aligned16(peers->v[r]))
     return fail(H3_ERR_ALIGN, "%s: this rank's q, k, v buffers must be 16-byte aligned", __func__);
+  if (qn_w || kn_w) {
+    H3_REQUIRE_PTR(qn_w);
+    H3_REQUIRE_PTR(kn_w);
+  }
   AttnProblem p;
   memset(&p, 0, sizeof(p));
+  p.qn_w = reinterpret_cast<const bf16*>(qn_w);
+  p.kn_w = reinterpret_cast<const bf16*>(kn_w);
   p.q = reinterpret_cast<const bf16*>(peers->q[r]);
   p.k = reinterpret_cast<const bf16*>(peers->k[r]);
   p.v = reinterpret_cast<const bf16*>(peers->v[r]);

@@ -131,18 +131,13 @@ __device__ __forceinline__ bool mbar_wait_spin_warp(uint64_t* bar, uint32_t pari
   return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity));
 }
 
-// Warp-uniform bounded waits in which lane 0 alone waits (polling with
-// test_wait, or suspending in try_wait) and the other lanes wait for its
-// verdict at a shuffle: one shared-memory probe per poll instead of 32.
-__device__ __forceinline__ bool mbar_wait_spin_lane0(uint64_t* bar, uint32_t parity) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait_spin(bar, parity) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-__device__ __forceinline__ bool mbar_wait_lane0(uint64_t* bar, uint32_t parity) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+// Warp-uniform form with a vote-first fast path: every lane probes the phase
+// once and the warp votes; only a warp that finds it incomplete enters the
+// bounded wait loop.  No lane leaves before the others (both votes take the
+// whole warp), and an already completed phase costs one probe and one vote.
+__device__ __forceinline__ bool mbar_wait_warp_fast(uint64_t* bar, uint32_t parity) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
 // ------------------------------------------------------------ clusters (CTA pairs)

@@ -132,7 +132,7 @@ def lib() -> ctypes.CDLL:
             "h3_sp_make_layout": (ci, [pd, pr, ci, ci, ctypes.POINTER(SPLayout), pr]),
             "h3_qkv_qknorm_mrope_sp": (ci, [pd, pr, ctypes.POINTER(SPLayout), vp, vp, vp, vp, vp, ci,
                                             ctypes.POINTER(SPPeers), vp]),
-            "h3_attention_sp": (ci, [pd, ctypes.POINTER(SPLayout), ctypes.POINTER(SPPeers), ci, vp]),
+            "h3_attention_sp": (ci, [pd, ctypes.POINTER(SPLayout), ctypes.POINTER(SPPeers), vp, vp, ci, vp]),
             "h3_text_refine": (ci, [pd, pr, vp, ci, ctypes.POINTER(ctypes.c_void_p), vp,
                                     ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockBuffers), ci, vp]),
         }
@@ -429,9 +429,10 @@ def h3_qkv_qknorm_mrope_sp(dims, shard, layout, xm, Wqkv, qn_w, kn_w, pos, peers
                                         _stream(stream)))
 
 
-def h3_attention_sp(dims, layout, peers: SPPeers, flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
-    _check(lib().h3_attention_sp(ctypes.byref(dims), ctypes.byref(layout), ctypes.byref(peers), flags,
-                                 _stream(stream)))
+def h3_attention_sp(dims, layout, peers: SPPeers, qn_w=None, kn_w=None, flags=H3_QK_NORM_ROPE_IN_QKV,
+                    stream=None):
+    _check(lib().h3_attention_sp(ctypes.byref(dims), ctypes.byref(layout), ctypes.byref(peers),
+                                 _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"), flags, _stream(stream)))
 
 
 def h3_text_refine(dims, ranges, x, mods: list, pos, weights: list, buffers: BlockBuffers,

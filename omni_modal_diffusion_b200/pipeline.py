@@ -72,7 +72,7 @@ class H3BlockStep:
         h3.h3_adaln_norm_modulate(d, r, self.x, mod, h3.H3_MSA, self.xm, stream=stream)
         h3.h3_qkv_qknorm_mrope(d, r, self.xm, W["Wqkv"], W["qn_w"], W["kn_w"], self.pos, self.q, self.k, self.v,
                                stream=stream)
-        h3.h3_attention(d, r, self.q, self.k, self.v, self.o, stream=stream)
+        h3.h3_attention(d, r, self.q, self.k, self.v, self.o, qn_w=W["qn_w"], kn_w=W["kn_w"], stream=stream)
         h3.h3_gated_residual(d, r, self.x, self.o, W["Wo"], mod, h3.H3_MSA, stream=stream)
         h3.h3_adaln_norm_modulate(d, r, self.x, mod, h3.H3_MLP, self.xm, stream=stream)
         h3.h3_ffn_swiglu(d, r, self.x, self.xm, W["Wgu"], W["Wd"], mod, self.ws, stream=stream)
@@ -149,11 +149,14 @@ class H3BlockStep:
         self.head_euler(lat_video, lat_audio, sig_video, sig_audio, stream=stream)
 
     # kernels launched by one step (for the launch count the bench reports)
-    def launches_per_step(self, e4m3: bool = False) -> int:
+    def launches_per_step(self, e4m3: bool = False, qk_e4m3: bool = False) -> int:
         r = self.ranges
         embed = (1 if r.count[2] > 0 else 0) + 1 + (1 if r.L_pad > r.L else 0) + sum(1 for c in r.count if c > 0)
-        # LN, QKV, attention, [quantise o,] out-projection, LN, FFN (2 GEMMs [+ quantise h])
-        block = 1 + 1 + 1 + 1 + 1 + 2 + (2 if e4m3 else 0)
+        # LN, QKV, attention (the split kernel + the general kernel's fixup
+        # launch; one kernel with e4m3 q, k), [quantise o,] out-projection,
+        # LN, FFN (2 GEMMs [+ quantise h])
+        attn = 1 if qk_e4m3 else 2
+        block = 1 + 1 + attn + 1 + 1 + 2 + (2 if e4m3 else 0)
         # head + Euler: LN, video head GEMM, audio head GEMM (Euler in their epilogues)
         head = 1 + (1 if r.count[2] > 0 else 0) + (1 if r.count[1] > 0 else 0)
         return embed + block + head
@@ -259,5 +262,6 @@ class H3Sampler:
 
     def launches_per_step(self) -> int:
         st = self.st
-        per_block = 9 if self.e4m3 else 7
-        return st.launches_per_step() - 7 + per_block * self.n_layers
+        qk8 = bool(self.flags & h3.H3_QK_E4M3)
+        per_block = (9 if self.e4m3 else 7) + (0 if qk8 else 1)
+        return st.launches_per_step() - 8 + per_block * self.n_layers

@@ -57,10 +57,13 @@ class SPRank:
         h3.h3_qkv_qknorm_mrope_sp(d, s, self.layout, self.xm, W["Wqkv"], W["qn_w"], W["kn_w"], self.pos,
                                   self.peers, stream=stream)
 
-    def phase_attention(self, stream=None):
+    def phase_attention(self, W=None, stream=None):
         """Attention for this rank's heads over all tokens, each output row
-        stored into its owner's o."""
-        h3.h3_attention_sp(self.dims, self.layout, self.peers, stream=stream)
+        stored into its owner's o (W: the block weights, whose Q/K norm
+        weights select the split-softmax kernel, as in the single-sequence
+        block)."""
+        qn, kn = (W["qn_w"], W["kn_w"]) if W is not None else (None, None)
+        h3.h3_attention_sp(self.dims, self.layout, self.peers, qn_w=qn, kn_w=kn, stream=stream)
 
     def phase_out_ffn(self, mod, W, stream=None):
         """The token-local rest of the block on this shard."""
@@ -92,7 +95,7 @@ def block_forward(ranks: list[SPRank], mod, W, barrier=None, stream=None):
     if barrier:
         barrier()
     for r in ranks:
-        r.phase_attention(stream)
+        r.phase_attention(W, stream)
     if barrier:
         barrier()
     for r in ranks:

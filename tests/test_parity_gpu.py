@@ -390,6 +390,77 @@ def test_attention_reference_moves(kind):
     assert np.all(got[L:] == 0)
 
 
+def _normalised(rng, H, Lp, w):
+    """Rows as the QKV call writes them: RMS-normalised, scaled by the norm
+    weight w, rounded to bf16."""
+    x = rng.standard_normal((H, Lp, 128))
+    return S.bf16_round((x / np.sqrt((x * x).mean(-1, keepdims=True) + 1e-6) * w).astype(np.float32))
+
+
+@pytest.mark.parametrize("L", [1, 64, 127, 128, 129, 3 * 128 + 5, 1000])
+def test_attention_split_normalised(L):
+    """Normalised q, k with their norm weights: the split-softmax kernel
+    (exponentials against the static bound, each row over two warps), down to
+    one key, a half-empty key tile and an odd query-tile count."""
+    H = 4
+    d = h3.make_dims(320, H, 896)
+    rg = h3.h3_make_ranges(L, 0, 0)
+    Lp = rg.L_pad
+    rng = np.random.default_rng(700 + L)
+    qn = S.bf16_round((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    kn = S.bf16_round((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    q, k = _normalised(rng, H, Lp, qn), _normalised(rng, H, Lp, kn)
+    v = S.bf16_round(rng.standard_normal((H, Lp, 128), dtype=np.float32))
+    for a in (q, k, v):
+        a[:, L:, :] = 0
+    o = torch.full((Lp, H * 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    h3.h3_attention(d, rg, *(to_dev_bf16(a, DEV) for a in (q, k, v)), o, qn_w=to_dev_bf16(qn, DEV),
+                    kn_w=to_dev_bf16(kn, DEV))
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    got = to_np(o)
+    ref = O.attention(*(a[:, :L, :].transpose(1, 0, 2).astype(np.float64) for a in (q, k, v)))
+    check_close(got[:L], ref, f"split attention L={L}")
+    assert np.all(got[L:] == 0)
+
+
+@pytest.mark.parametrize("kind", ["far_above", "far_below", "wide_bound"])
+def test_attention_split_falls_back(kind):
+    """Norm weights given but the bound does not hold, or is too wide: the
+    CTAs concerned are recomputed by the general kernel and the result is the
+    oracle's.  far_above: some keys 30x longer than normalised rows (scores
+    far above the bound); far_below: every key opposite to every query and 10x
+    longer (every p would flush to 0); wide_bound: norm weights near 2.5
+    (scores up to +-100 in log2 units, past the fp32 range of the exponentials
+    against the bound)."""
+    H, L = 4, 1000
+    d = h3.make_dims(320, H, 896)
+    rg = h3.h3_make_ranges(L, 0, 0)
+    Lp = rg.L_pad
+    rng = np.random.default_rng({"far_above": 11, "far_below": 12, "wide_bound": 13}[kind])
+    scale = 2.5 if kind == "wide_bound" else 1.0
+    qn = S.bf16_round((scale * (1 + 0.05 * rng.standard_normal(128))).astype(np.float32))
+    kn = S.bf16_round((scale * (1 + 0.05 * rng.standard_normal(128))).astype(np.float32))
+    q, k = _normalised(rng, H, Lp, qn), _normalised(rng, H, Lp, kn)
+    if kind == "far_above":
+        k[:, 3 * 128 + 64: 4 * 128] = S.bf16_round(30 * k[:, 3 * 128 + 64: 4 * 128])
+    elif kind == "far_below":
+        q[:] = q[:, :1, :]
+        k[:] = S.bf16_round((-10 * q[:, :1, :]).astype(np.float32))
+    v = S.bf16_round(rng.standard_normal((H, Lp, 128), dtype=np.float32))
+    for a in (q, k, v):
+        a[:, L:, :] = 0
+    o = torch.empty(Lp, H * 128, dtype=torch.bfloat16, device=DEV)
+    h3.h3_attention(d, rg, *(to_dev_bf16(a, DEV) for a in (q, k, v)), o, qn_w=to_dev_bf16(qn, DEV),
+                    kn_w=to_dev_bf16(kn, DEV))
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    got = to_np(o)
+    ref = O.attention(*(a[:, :L, :].transpose(1, 0, 2).astype(np.float64) for a in (q, k, v)))
+    check_close(got[:L], ref, f"split attention fallback ({kind})")
+    assert np.all(got[L:] == 0)
+
+
 # ---------------------------------------------------------------- full sizes, sampled outputs
 
 FULL = [S.WORKLOADS["768sq_2s"], S.WORKLOADS["768x1344_5s"]]
@@ -429,11 +500,17 @@ def test_full_length_attention_sampled_rows(L, H):
     rg = h3.h3_make_ranges(L, 0, 0)
     Lp = rg.L_pad
     rng = np.random.default_rng(L)
-    qkv = [S.bf16_round(rng.standard_normal((H, Lp, 128), dtype=np.float32)) for _ in range(3)]
+    # normalised q, k with their norm weights (the split-softmax kernel, as the
+    # block runs it)
+    qn = S.bf16_round((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    kn = S.bf16_round((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    qkv = [_normalised(rng, H, Lp, qn), _normalised(rng, H, Lp, kn),
+           S.bf16_round(rng.standard_normal((H, Lp, 128), dtype=np.float32))]
     for a in qkv:
         a[:, L:, :] = 0
     o = torch.empty(Lp, H * 128, dtype=torch.bfloat16, device=DEV)
-    h3.h3_attention(d, rg, *(to_dev_bf16(a, DEV) for a in qkv), o)
+    h3.h3_attention(d, rg, *(to_dev_bf16(a, DEV) for a in qkv), o, qn_w=to_dev_bf16(qn, DEV),
+                    kn_w=to_dev_bf16(kn, DEV))
     rows = _sample_rows(L, 48, seed=L)
     got = to_np(o[torch.from_numpy(rows).to(DEV)])
     q, k, v = (a[:, :L, :].transpose(1, 0, 2) for a in qkv)
