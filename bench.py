@@ -98,11 +98,11 @@ TRAFFIC = {
     # the same four launches with e4m3 operands (2.679 GB / 4)
     ("768sq_2s", "gemm_tc_kernel<e4m3>"): 0.670e9,
     # one attention launch at 124,016 tokens: DRAM read + write of a 2-head
-    # launch (495.6 MB + 59.8 MB) times 28 for the 56 heads (heads are
+    # launch (493.0 MB + 60.3 MB) times 28 for the 56 heads (heads are
     # independent CTAs, scheduled head after head, so the traffic grows with
     # them); q, k, v, o alone are 7.11 GB, the rest is K and V re-read by
     # CTAs that started at different times
-    ("768x1792_15s", "attention_split_kernel"): 15.55e9,
+    ("768x1792_15s", "attention_split_kernel"): 15.49e9,
 }
 
 

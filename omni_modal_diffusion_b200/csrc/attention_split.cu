@@ -16,6 +16,13 @@
 //   Warps 2-17   softmax: tile t = (w - 2) / 8, key half hf = ((w - 2) / 4) % 2,
 //                lane quarter w % 4 (the quarter a warp may access in TMEM)
 //
+// The MMA warp holds one wait on each tile's path from P to P V: the tile's
+// eight softmax warps arrive on one barrier, and the waits for V(j) and
+// K(j + 1), loaded a step or more earlier, come before the wait for tile 0's
+// P.  Every extra wait there showed in the time (a barrier per key half,
+// the V and K waits between the P V and S MMAs: 3% slower; a barrier per
+// 32-key chunk: 25% slower).
+//
 // The two halves of a row cannot move a softmax reference independently (O
 // accumulates both halves' P V against one reference), and agreeing on it
 // every key tile would put a handshake on each tile's critical path.  So
@@ -43,16 +50,7 @@ using attn_detail::TILE_BYTES;
 using attn_detail::TMEM_COLS;
 
 constexpr int NUM_THREADS = 18 * 32;
-// Order of the MMA warp's waits and stage releases: 1 puts every wait and
-// commit that is not on a P -> P V path where the warp waits for P anyway
-// (V(j) before tile 0's first P half, K(j + 1) after tile 0's first P V half,
-// the releases of K(j) and V(j - 1) after that half; needs a third V stage);
-// 0 waits for V and K right before the MMAs that read them and releases
-// each stage after its last MMA.
-#ifndef H3_ATTN_SPLIT_ORDER
-#define H3_ATTN_SPLIT_ORDER 0
-#endif
-constexpr int SVS = H3_ATTN_SPLIT_ORDER ? 3 : 2;  // V stages
+constexpr int SVS = 2;                       // V stages
 constexpr int SQ = 0;                       // 2 query tiles
 constexpr int SK = SQ + 2 * TILE_BYTES;     // 2 stages
 constexpr int SV = SK + 2 * TILE_BYTES;     // SVS stages
@@ -100,12 +98,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* v_empty = bars + 8;   // [SVS]
   uint64_t* s_full = bars + 11;   // [2] per query tile
   uint64_t* o_final = bars + 13;  // [2] per query tile
-  uint64_t* p_full = bars + 15;   // [2 tiles][2 halves]: 4 warp arrivals each
-  uint64_t* drain = bars + 19;
-  uint64_t* sums_done = bars + 20;  // [2] every softmax warp has written its row sums / its low-side verdict
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
-  float* bound = reinterpret_cast<float*>(bars + 23);
-  int* cta_bad = reinterpret_cast<int*>(bars + 24);
+  uint64_t* p_full = bars + 15;   // [2] per query tile: its 8 softmax warps' arrivals
+  uint64_t* drain = bars + 17;
+  uint64_t* sums_done = bars + 18;  // [2] every softmax warp has written its row sums / its low-side verdict
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  float* bound = reinterpret_cast<float*>(bars + 21);
+  int* cta_bad = reinterpret_cast<int*>(bars + 22);
   float* lsum = reinterpret_cast<float*>(smem + SSUM + (((L + TILE - 1) / TILE) & 1) * TILE_BYTES);  // [t][hf][row]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -125,8 +123,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&k_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&o_final[s], 1);
-      mbar_init(&p_full[2 * s], 4);
-      mbar_init(&p_full[2 * s + 1], 4);
+      mbar_init(&p_full[s], 8);
     }
     for (int s = 0; s < SVS; ++s) {
       mbar_init(&v_full[s], 1);
@@ -214,46 +211,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       umma_commit(&s_full[t]);
     };
-    // O_t += P_t V_j for keys [64 hf, 64 hf + 64): that half's P sits in
-    // TMEM columns [64 hf, 64 hf + 32) of the tile's S region
-    auto issue_pv_half = [&](int t, int j, int hf) {
+    // O_t += P_t V_j: the P of keys [64 hf, 64 hf + 64) sits in TMEM columns
+    // [64 hf, 64 hf + 32) of the tile's S region (written by that half's warps)
+    auto issue_pv = [&](int t, int j) {
       const uint64_t vd = v_desc + (uint64_t)(((j % SVS) * TILE_BYTES) >> 4);
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int kk = hf * 4 + k4;
-        umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + hf * 64 + k4 * 8,
+      for (int kk = 0; kk < 8; ++kk)
+        umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + (kk >> 2) * 64 + (kk & 3) * 8,
                          vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j | kk) != 0 ? 1u : 0u);
-      }
     };
     bool ok = mbar_wait_warp(q_full, 0) && mbar_wait_warp(&k_full[0], 0);
-#if H3_ATTN_SPLIT_ORDER
-    if (ok) {
-      tc_fence_after();
-      issue_s(0, 0);
-      if (two) issue_s(1, 0);
-    }
-    for (int j = 0; j < nkv && ok; ++j) {
-      const bool more = j + 1 < nkv;
-      if (!mbar_wait_warp_fast(&v_full[j % SVS], (j / SVS) & 1)) { ok = false; break; }
-      for (int t = 0; t < nt; ++t) {
-        if (!mbar_wait_warp_fast(&p_full[2 * t], j & 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv_half(t, j, 0);
-        if (t == 0) {
-          umma_commit(&k_empty[j & 1]);                     // K(j): its last S MMA was issued a step ago
-          if (j > 0) umma_commit(&v_empty[(j - 1) % SVS]);  // V(j - 1): its last P V likewise
-          if (more && !mbar_wait_warp_fast(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
-        }
-        if (!mbar_wait_warp_fast(&p_full[2 * t + 1], j & 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv_half(t, j, 1);
-        if (more)
-          issue_s(t, j + 1);
-        else
-          umma_commit(&o_final[t]);
-      }
-    }
-#else
     if (ok) {
       tc_fence_after();
       issue_s(0, 0);
@@ -262,19 +229,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int j = 0; j < nkv && ok; ++j) {
       const bool more = j + 1 < nkv;
+      // V(j) and K(j + 1) were requested a step or more ago: check them before
+      // waiting for tile 0's P, so that each tile's P -> P V path holds one
+      // wait (measured 3% faster than waiting for each just before its MMAs)
+      ok = mbar_wait_warp(&v_full[j % SVS], (j / SVS) & 1) &&
+           (!more || mbar_wait_warp(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1));
       for (int t = 0; t < nt && ok; ++t) {
-        for (int hf = 0; hf < 2; ++hf) {
-          if (!mbar_wait_warp(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
-          if (t == 0 && hf == 0 && !mbar_wait_warp(&v_full[j % SVS], (j / SVS) & 1)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv_half(t, j, hf);
-        }
-        if (!ok) break;
+        if (!mbar_wait_warp(&p_full[t], j & 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(t, j);
         if (more) {
-          if (t == 0) {
-            if (!mbar_wait_warp(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-          }
           issue_s(t, j + 1);
           if (t == nt - 1) umma_commit(&k_empty[(j + 1) & 1]);
         } else {
@@ -283,7 +247,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       umma_commit(&v_empty[j % SVS]);
     }
-#endif
     drain_mmas(drain);
   } else if (((warp - 2) >> 3) < nt) {
     const int t = (warp - 2) >> 3;         // query tile
@@ -345,7 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[2 * t + hf]);
+      if (lane == 0) mbar_arrive(&p_full[t]);
       bad |= !(hs <= HALF_SUM_LIMIT);
       l_part += hs;
     }

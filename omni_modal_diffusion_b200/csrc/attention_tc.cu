@@ -89,6 +89,10 @@ constexpr float P_HALF_SUM_LIMIT = 65536.0f;
 #ifndef H3_ATTN_MMA_SPIN
 #define H3_ATTN_MMA_SPIN 0
 #endif
+// 1: the MMA warp checks V(j) and K(j + 1) before waiting for tile 0's P
+#ifndef H3_ATTN_VK_AHEAD
+#define H3_ATTN_VK_AHEAD 0
+#endif
 #if H3_ATTN_MMA_SPIN
 #define MMA_WAIT_WARP mbar_wait_spin_warp
 #else
@@ -277,19 +281,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int j = 0; j < nkv && ok; ++j) {
       const bool more = j + 1 < nkv;
+#if H3_ATTN_VK_AHEAD
+      // V(j) and K(j + 1) were requested a step or more ago: checked before
+      // the wait for tile 0's P, off the P -> P V path
+      ok = MMA_WAIT_WARP(&v_full[j % VS], (j / VS) & 1) &&
+           (!more || MMA_WAIT_WARP(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1));
+#endif
       for (int t = 0; t < nt && ok; ++t) {
         // P is released in two halves: PV on keys [0, 64) runs while the
         // softmax warps still take the second half's exponentials
         for (int hf = 0; hf < 2; ++hf) {
           if (!MMA_WAIT_WARP(&p_full[2 * t + hf], j & 1)) { ok = false; break; }
-          if (t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j % VS], (j / VS) & 1)) { ok = false; break; }
+          if (!H3_ATTN_VK_AHEAD && t == 0 && hf == 0 && !MMA_WAIT_WARP(&v_full[j % VS], (j / VS) & 1)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           issue_pv_half(t, j, hf);
           if (hf == 0) umma_commit(&pv0_done[t]);
         }
         if (!ok) break;
         if (more) {
-          if (t == 0) {
+          if (!H3_ATTN_VK_AHEAD && t == 0) {
             if (!MMA_WAIT_WARP(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
           }

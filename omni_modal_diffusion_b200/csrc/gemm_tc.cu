@@ -20,6 +20,10 @@
 
 namespace h3 {
 
+#ifndef H3_GEMM_HALF_N
+#define H3_GEMM_HALF_N 1
+#endif
+
 namespace gemm_detail {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_STAGE_BYTES = BM * BK * 2;  // 16 KB
@@ -428,6 +432,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_tiles = m_tiles * p.n_tiles;
   const int num_kb = (p.K + KSTEP - 1) / KSTEP;
   const bool swiglu = e.mode == EPI_SWIGLU;
+  // A narrow output (the heads: 96 or fewer columns) takes one 128-row B box
+  // and N = 128 MMAs, half the tensor work of a 256-wide tile: these GEMMs
+  // stream A from HBM and have no use for the other half
+  const bool half_n = H3_GEMM_HALF_N && !F8 && p.n_tiles == 1 && p.N_b_rows <= 128 &&
+                      (e.mode == EPI_STORE_F32 || e.mode == EPI_UNPATCH);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -442,10 +451,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int b1 = b0 + p.b_second_half_off;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          mbar_arrive_expect_tx(&full[stage], half_n ? STAGE_BYTES - B_STAGE_BYTES / 2 : STAGE_BYTES);
           tma_load_2d(smA + stage * A_STAGE_BYTES, &tmA, &full[stage], kb * KSTEP, mt * BM);
           tma_load_2d(smB + stage * B_STAGE_BYTES, &tmB, &full[stage], kb * KSTEP, b0);
-          tma_load_2d(smB + stage * B_STAGE_BYTES + B_STAGE_BYTES / 2, &tmB, &full[stage], kb * KSTEP, b1);
+          if (!half_n)
+            tma_load_2d(smB + stage * B_STAGE_BYTES + B_STAGE_BYTES / 2, &tmB, &full[stage], kb * KSTEP, b1);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -454,7 +464,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // The whole warp runs the issue loop, converged; one elected lane issues.
-    const uint32_t idesc = F8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, BN, false);
+    const uint32_t idesc = F8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, half_n ? 128 : BN, false);
     // descriptors computed once; per MMA only the start address moves
     // (16-byte units: a 32-byte K step is +2)
     const uint64_t a_desc0 = sdesc_sw128(smem_u32(smA), 16, 1024);
