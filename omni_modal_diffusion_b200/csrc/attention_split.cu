@@ -37,6 +37,13 @@
 // B > 60 leaves a NaN sentinel in its first output element instead of its
 // rows, and a second launch of attention_tc_kernel recomputes exactly those
 // CTAs with its moving reference.
+//
+// QK8: Q and K arrive as e4m3 codes of q * 448 / (sqrt(128) max|qn_w|) and
+// k * 448 / (sqrt(128) max|kn_w|) (the QKV epilogue's H3_QK_E4M3 output); S
+// is four kind::f8f6f4 MMAs per tile and its dequantisation folds into the
+// exponent scale.  Rounding q and k to e4m3 (3 mantissa bits) moves each
+// element by at most 2^-4 of itself, so the bound takes the factor
+// (1 + 2^-4)^2 = 1.129: B = 16.32 * 1.14 max|qn_w| max|kn_w|.
 #include "h3_internal.cuh"
 #include "ptx.cuh"
 
@@ -50,17 +57,23 @@ using attn_detail::TILE_BYTES;
 using attn_detail::TMEM_COLS;
 
 constexpr int NUM_THREADS = 18 * 32;
-constexpr int SVS = 2;                       // V stages
-constexpr int SQ = 0;                       // 2 query tiles
-constexpr int SK = SQ + 2 * TILE_BYTES;     // 2 stages
-constexpr int SV = SK + 2 * TILE_BYTES;     // SVS stages
-constexpr int SBAR = SV + SVS * TILE_BYTES;
-constexpr int BYTES = SBAR + 256 + 1024;
-// [2 tiles][2 halves][128 rows] row sums, written after a warp's key loop:
-// over the K stage that held K(nkv - 2), whose last S MMA completed before
-// any tile's last S (the other stage may still feed the other tile's last S)
-constexpr int SSUM = SK;
-static_assert(BYTES <= 232448, "shared memory per CTA");
+constexpr int SVS = 2;  // V stages
+template <bool QK8>
+struct SLayout {
+  static constexpr int QK_TILE = QK8 ? TILE_BYTES / 2 : TILE_BYTES;  // a Q or K tile (e4m3: 128-byte rows)
+  static constexpr int SQ = 0;                                        // 2 query tiles
+  static constexpr int SK = SQ + 2 * QK_TILE;                         // 2 stages
+  static constexpr int SV = SK + 2 * QK_TILE;                         // SVS stages
+  static constexpr int SBAR = SV + SVS * TILE_BYTES;
+  static constexpr int BYTES = SBAR + 256 + 1024;
+  // [2 tiles][2 halves][128 rows] row sums (2 KB), written after a warp's key
+  // loop: over the K stage that held K(nkv - 2), whose last S MMA completed
+  // before any tile's last S (the other stage may still feed the other
+  // tile's last S)
+  static constexpr int SSUM = SK;
+  static_assert(BYTES <= 232448, "shared memory per CTA");
+  static_assert(QK_TILE >= 2 * 2 * 128 * 4, "row sums fit in a K stage");
+};
 constexpr float B_MAX = 60.0f;              // largest bound whose p stay >= 2^-120
 constexpr float HALF_SUM_LIMIT = 4294967296.0f;  // 2^32: a key half above it breaks the bound
 
@@ -80,10 +93,13 @@ __device__ __forceinline__ bf16* sentinel_ptr(const AttnOut& out, int grow, int 
   return out.shard[owner] + (long)(grow - owner * out.L_shard) * out.ld + (out.head0 + h) * 128;
 }
 
+template <bool QK8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attention_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnOut out, int H,
                            int L, int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w) {
+  using Y = SLayout<QK8>;
+  constexpr int SQ = Y::SQ, SK = Y::SK, SV = Y::SV, SBAR = Y::SBAR, SSUM = Y::SSUM, QK_TILE = Y::QK_TILE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -104,7 +120,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   float* bound = reinterpret_cast<float*>(bars + 21);
   int* cta_bad = reinterpret_cast<int*>(bars + 22);
-  float* lsum = reinterpret_cast<float*>(smem + SSUM + (((L + TILE - 1) / TILE) & 1) * TILE_BYTES);  // [t][hf][row]
+  float* qk_scale = reinterpret_cast<float*>(bars + 23);  // QK8: dequantisation of S
+  float* lsum = reinterpret_cast<float*>(smem + SSUM + (((L + TILE - 1) / TILE) & 1) * QK_TILE);  // [t][hf][row]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = L_pad / TILE;
@@ -154,8 +171,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
       mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
     }
-    // 128 mq mk (1 + 2^-9)^2 log2(e) / sqrt(128), with a 1% margin
-    if (lane == 0) *bound = 16.3219f * 1.01f * mq * mk;
+    // 128 mq mk (1 + 2^-9)^2 log2(e) / sqrt(128), with a 1% margin (QK8:
+    // times the e4m3 factor 1.129, with a 1% margin)
+    if (lane == 0) {
+      *bound = 16.3219f * (QK8 ? 1.14f : 1.01f) * mq * mk;
+      if (QK8) *qk_scale = ((11.3137085f * mq) / 448.0f) * ((11.3137085f * mk) / 448.0f);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -170,19 +191,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (threadIdx.x == 0) *sentinel_ptr(out, qt0 * TILE, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
   } else if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, nt * TILE_BYTES);
+      mbar_arrive_expect_tx(q_full, nt * QK_TILE);
       for (int t = 0; t < nt; ++t) {
         const int qrow = row0 + (t == 0 ? qt0 : qt1) * TILE;
-        tma_load_2d(sQ + t * TILE_BYTES, &tmQ, q_full, 0, qrow);
-        tma_load_2d(sQ + t * TILE_BYTES + HALF_BYTES, &tmQ, q_full, 64, qrow);
+        tma_load_2d(sQ + t * QK_TILE, &tmQ, q_full, 0, qrow);
+        if (!QK8) tma_load_2d(sQ + t * QK_TILE + HALF_BYTES, &tmQ, q_full, 64, qrow);
       }
       long long k_issued = 0, v_issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int st = j & 1;
         if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1)) break;
-        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
-        tma_load_2d(sK + st * TILE_BYTES, &tmK, &k_full[st], 0, row0 + j * TILE);
-        tma_load_2d(sK + st * TILE_BYTES + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
+        mbar_arrive_expect_tx(&k_full[st], QK_TILE);
+        tma_load_2d(sK + st * QK_TILE, &tmK, &k_full[st], 0, row0 + j * TILE);
+        if (!QK8) tma_load_2d(sK + st * QK_TILE + HALF_BYTES, &tmK, &k_full[st], 64, row0 + j * TILE);
         ++k_issued;
         const int sv = j % SVS;
         if (!mbar_wait(&v_empty[sv], ((j / SVS) & 1) ^ 1)) break;
@@ -196,18 +217,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_loads(v_full, SVS, v_issued);
     }
   } else if (warp == 1) {
-    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+    const uint32_t idesc_s = QK8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);  // V is MN-major
     const uint64_t q_desc = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t k_desc = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t v_desc = sdesc_sw128(smem_u32(sV), HALF_BYTES, 1024);
     auto issue_s = [&](int t, int j) {
-      const uint64_t qd = q_desc + (uint64_t)((t * TILE_BYTES) >> 4);
-      const uint64_t kd = k_desc + (uint64_t)(((j & 1) * TILE_BYTES) >> 4);
+      const uint64_t qd = q_desc + (uint64_t)((t * QK_TILE) >> 4);
+      const uint64_t kd = k_desc + (uint64_t)(((j & 1) * QK_TILE) >> 4);
+      if constexpr (QK8) {
+        // one 128-byte row per token: four MMAs of K = 32 codes (32 bytes)
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-        umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk)
+          umma_e4m3(tmem + t * 256, qd + (uint64_t)(kk * 2), kd + (uint64_t)(kk * 2), idesc_s, kk != 0 ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+          umma_bf16(tmem + t * 256, qd + off, kd + off, idesc_s, kk != 0 ? 1u : 0u);
+        }
       }
       umma_commit(&s_full[t]);
     };
@@ -256,7 +284,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = tmem + ((uint32_t)(qw * 32) << 16) + t * 256;
     const uint32_t tH = tS + hf * 64;      // this warp's 64 score columns; its P goes to the first 32
     const uint32_t tO = tS + 128;
-    const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+    // QK8: the dequantisation of S folds into the scale; an all-zero norm
+    // weight (every code 0, S = 0) is raised to a tiny positive scale so
+    // masked keys (-inf) still give 0 and not 0 * inf = NaN
+    const float sl2 = QK8 ? fmaxf(scale_log2 * *qk_scale, 1e-30f) : scale_log2;
+    const uint64_t sc2 = f2_pack(sl2, sl2);
     const uint64_t nb2 = f2_pack(-B, -B);
     float l_part = 0.f;
     bool bad = false;
@@ -368,13 +400,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 cudaError_t launch_attention_split(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                    const attn_detail::AttnOut& out, dim3 grid, int H, int L, int L_pad,
-                                   float scale_log2, const bf16* qn_w, const bf16* kn_w, cudaStream_t stream) {
-  static unsigned long long attr_done = 0;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(attn_split::attention_split_kernel),
-                                   attn_split::BYTES, &attr_done);
+                                   float scale_log2, const bf16* qn_w, const bf16* kn_w, bool qk8,
+                                   cudaStream_t stream) {
+  static unsigned long long attr_done[2] = {0, 0};
+  const void* kfn = qk8 ? reinterpret_cast<const void*>(attn_split::attention_split_kernel<true>)
+                        : reinterpret_cast<const void*>(attn_split::attention_split_kernel<false>);
+  cudaError_t e = ensure_smem_attr(kfn, qk8 ? attn_split::SLayout<true>::BYTES : attn_split::SLayout<false>::BYTES,
+                                   &attr_done[qk8 ? 1 : 0]);
   if (e != cudaSuccess) return e;
-  attn_split::attention_split_kernel<<<grid, attn_split::NUM_THREADS, attn_split::BYTES, stream>>>(
-      tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w);
+  if (qk8)
+    attn_split::attention_split_kernel<true><<<grid, attn_split::NUM_THREADS, attn_split::SLayout<true>::BYTES, stream>>>(
+        tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w);
+  else
+    attn_split::attention_split_kernel<false>
+        <<<grid, attn_split::NUM_THREADS, attn_split::SLayout<false>::BYTES, stream>>>(tq, tk, tv, out, H, L, L_pad,
+                                                                                       scale_log2, qn_w, kn_w);
   return cudaGetLastError();
 }
 

@@ -153,9 +153,9 @@ class H3BlockStep:
         r = self.ranges
         embed = (1 if r.count[2] > 0 else 0) + 1 + (1 if r.L_pad > r.L else 0) + sum(1 for c in r.count if c > 0)
         # LN, QKV, attention (the split kernel + the general kernel's fixup
-        # launch; one kernel with e4m3 q, k), [quantise o,] out-projection,
-        # LN, FFN (2 GEMMs [+ quantise h])
-        attn = 1 if qk_e4m3 else 2
+        # launch, bf16 or e4m3 q, k), [quantise o,] out-projection, LN, FFN
+        # (2 GEMMs [+ quantise h])
+        attn = 2
         block = 1 + 1 + attn + 1 + 1 + 2 + (2 if e4m3 else 0)
         # head + Euler: LN, video head GEMM, audio head GEMM (Euler in their epilogues)
         head = 1 + (1 if r.count[2] > 0 else 0) + (1 if r.count[1] > 0 else 0)
@@ -262,6 +262,5 @@ class H3Sampler:
 
     def launches_per_step(self) -> int:
         st = self.st
-        qk8 = bool(self.flags & h3.H3_QK_E4M3)
-        per_block = (9 if self.e4m3 else 7) + (0 if qk8 else 1)
+        per_block = (9 if self.e4m3 else 7) + 1  # attention: split kernel + fixup launch
         return st.launches_per_step() - 8 + per_block * self.n_layers

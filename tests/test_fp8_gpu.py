@@ -287,6 +287,38 @@ def test_attention_e4m3_qk(L):
     assert np.all(got[L:] == 0)
 
 
+def test_attention_e4m3_qk_wide_bound_falls_back():
+    """Norm weights near 2.5 put the static score bound of the split kernel
+    on e4m3 codes (16.32 * 1.14 max|qn_w| max|kn_w| ~ 116) above the 60 it
+    accepts: every CTA leaves its sentinel and the general kernel recomputes
+    it with its moving softmax reference; the result is the same attention."""
+    H, L = 4, 389
+    d = h3.make_dims(320, H, 896)
+    rg = h3.h3_make_ranges(L, 0, 0)
+    Lp = rg.L_pad
+    rng = np.random.default_rng(311)
+    qn = S.bf16_round((2.5 * (1 + 0.05 * rng.standard_normal(128))).astype(np.float32))
+    kn = S.bf16_round((2.5 * (1 + 0.05 * rng.standard_normal(128))).astype(np.float32))
+    def normed(wn):
+        x = rng.standard_normal((H, Lp, 128))
+        return x / np.sqrt((x ** 2).mean(-1, keepdims=True)) * wn
+    q8, k8 = F8.quantize_qk(normed(qn), qn), F8.quantize_qk(normed(kn), kn)
+    v = S.bf16_round(rng.standard_normal((H, Lp, 128), dtype=np.float32))
+    for a in (q8, k8):
+        a[:, L:, :] = 0
+    v[:, L:, :] = 0
+    o = torch.empty(Lp, H * 128, dtype=torch.bfloat16, device=DEV)
+    h3.h3_attention(d, rg, _u8(q8), _u8(k8), to_dev_bf16(v, DEV), o, qn_w=to_dev_bf16(qn, DEV),
+                    kn_w=to_dev_bf16(kn, DEV), flags=h3.H3_QK_NORM_ROPE_IN_QKV | h3.H3_QK_E4M3)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    got = to_np(o)
+    qd, kd = F8.dequantize_qk(q8, qn), F8.dequantize_qk(k8, kn)
+    ref = O.attention(*(a[:, :L, :].transpose(1, 0, 2).astype(np.float64) for a in (qd, kd, v)))
+    check_close(got[:L], ref, "e4m3-QK attention, wide bound (recomputed by the general kernel)")
+    assert np.all(got[L:] == 0)
+
+
 def test_e4m3_qk_zero_norm_weight():
     """An all-zero q norm weight: every q element is 0, so its e4m3 codes are
     0 (inverse scale 0, not 0 * inf) and attention is the plain average of v
