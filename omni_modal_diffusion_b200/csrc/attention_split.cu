@@ -58,15 +58,6 @@ using attn_detail::TMEM_COLS;
 
 constexpr int NUM_THREADS = 18 * 32;
 constexpr int SVS = 2;  // V stages
-// TMEM traffic of a softmax warp per key tile: 0 two 32-column loads, each
-// waited for, and two 16-column P stores; 1 both loads before one wait and
-// one 32-column P store (fewer waits and instructions through the
-// sub-partition's memory-instruction queue, which the MMA warp's stalled
-// issues also occupy); 2 the same for the warps of lane quarter 1 only (the
-// MMA warp's sub-partition)
-#ifndef H3_ATTN_SPLIT_WIDE
-#define H3_ATTN_SPLIT_WIDE 0
-#endif
 template <bool QK8>
 struct SLayout {
   static constexpr int QK_TILE = QK8 ? TILE_BYTES / 2 : TILE_BYTES;  // a Q or K tile (e4m3: 128-byte rows)
@@ -324,32 +315,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const int valid = L - j * TILE - hf * 64;  // this half's keys [0, valid) are real
-#if H3_ATTN_SPLIT_WIDE
-      if (H3_ATTN_SPLIT_WIDE == 1 || qw == 1) {
-        float s1[32], s2[32];
-        uint32_t pk[32];
-        tmem_ld32(tH, reinterpret_cast<uint32_t*>(s1));
-        tmem_ld32(tH + 32, reinterpret_cast<uint32_t*>(s2));
-        tmem_wait_ld();
-        if (valid < 64) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (c >= valid) s1[c] = -INFINITY;
-            if (c + 32 >= valid) s2[c] = -INFINITY;
-          }
-        }
-        float hs = exp32(s1, pk);
-        hs += exp32(s2, pk + 16);
-        tmem_st32(tH, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[t]);
-        bad |= !(hs <= HALF_SUM_LIMIT);
-        l_part += hs;
-        continue;
-      }
-#endif
       float s[32];
       uint32_t pkA[16], pkB[16];
       tmem_ld32(tH, reinterpret_cast<uint32_t*>(s));
