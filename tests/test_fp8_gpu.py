@@ -287,6 +287,46 @@ def test_attention_e4m3_qk(L):
     assert np.all(got[L:] == 0)
 
 
+def test_full_length_attention_e4m3_qk_sampled_rows():
+    """e4m3 q, k codes at the longest packed length (124,016 tokens, 2 heads:
+    heads are independent CTAs), sampled query rows (with the first, middle
+    and last rows) against the oracle's attention on the dequantised codes
+    over all keys."""
+    H, L = 2, 124016
+    d = h3.make_dims(5376, H, 14336)
+    rg = h3.h3_make_ranges(L, 0, 0)
+    Lp = rg.L_pad
+    rng = np.random.default_rng(L + 8)
+    qn = S.bf16_round((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    kn = S.bf16_round((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    def codes(wn):
+        # the codes are inputs to both sides, so any correct rounding serves:
+        # torch's CPU float8_e4m3fn conversion (the one the oracle's encoder
+        # is pinned to) instead of the oracle's slower search at this size
+        x = rng.standard_normal((H, Lp, 128))
+        x = x / np.sqrt((x ** 2).mean(-1, keepdims=True)) * wn
+        inv, _ = F8.qk_code_scale(wn)
+        xs = torch.from_numpy((x * np.float64(inv)).astype(np.float32))
+        return xs.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    q8, k8 = codes(qn), codes(kn)
+    v = S.bf16_round(rng.standard_normal((H, Lp, 128), dtype=np.float32))
+    for a in (q8, k8):
+        a[:, L:, :] = 0
+    v[:, L:, :] = 0
+    o = torch.empty(Lp, H * 128, dtype=torch.bfloat16, device=DEV)
+    h3.h3_attention(d, rg, _u8(q8), _u8(k8), to_dev_bf16(v, DEV), o, qn_w=to_dev_bf16(qn, DEV),
+                    kn_w=to_dev_bf16(kn, DEV), flags=h3.H3_QK_NORM_ROPE_IN_QKV | h3.H3_QK_E4M3)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    rows = np.unique(np.concatenate([S.random_rows(L, 48, seed=L + 8), [0, 1, L // 2, L - 2, L - 1]]))
+    got = to_np(o[torch.from_numpy(rows).to(DEV)])
+    qd, kd = F8.dequantize_qk(q8[:, :L], qn), F8.dequantize_qk(k8[:, :L], kn)
+    q, k, vv = (a.transpose(1, 0, 2).astype(np.float64) for a in (qd, kd, v[:, :L]))
+    ref = O.attention_rows(q[rows], k, vv)
+    check_close(got, ref, "e4m3-QK attention L=124016 rows")
+    assert float(o[L:].float().abs().max()) == 0.0
+
+
 def test_attention_e4m3_qk_wide_bound_falls_back():
     """Norm weights near 2.5 put the static score bound of the split kernel
     on e4m3 codes (16.32 * 1.14 max|qn_w| max|kn_w| ~ 116) above the 60 it
