@@ -217,6 +217,8 @@ def run_ours(args, w):
          "Wo": randn(w.D, w.I, std=0.02), "Wgu": randn(2 * w.F, w.D, std=0.02), "Wd": randn(w.D, w.F, std=0.02),
          "W_vhead": randn(4 * w.C_lat, w.D, std=0.02), "W_ahead": randn(w.C_audio, w.D, std=0.02)}
     st = H3BlockStep(w, device=dev, weights=W)
+    if getattr(args, "qk_prologue", False):
+        st.qk_flags = 0  # raw q, k; norm + RoPE in attention's prologue
     L, Lp = st.ranges.L, st.ranges.L_pad
     text = randn(w.n_text, w.D_text)
     video = randn(w.T_lat, w.H_lat, w.W_lat, w.C_lat)
@@ -238,9 +240,13 @@ def run_ours(args, w):
         mark(0, 0); st.embed(text, video, audio); mark(0, 1)
         mark(1, 0); h3.h3_adaln_norm_modulate(d, r, st.x, mod, h3.H3_MSA, st.xm); mark(1, 1)
         mark(2, 0)
-        h3.h3_qkv_qknorm_mrope(d, r, st.xm, st.W["Wqkv"], st.W["qn_w"], st.W["kn_w"], st.pos, st.q, st.k, st.v)
+        h3.h3_qkv_qknorm_mrope(d, r, st.xm, st.W["Wqkv"], st.W["qn_w"], st.W["kn_w"], st.pos, st.q, st.k, st.v,
+                               flags=st.qk_flags)
         mark(2, 1)
-        mark(3, 0); h3.h3_attention(d, r, st.q, st.k, st.v, st.o, qn_w=st.W["qn_w"], kn_w=st.W["kn_w"]); mark(3, 1)
+        mark(3, 0)
+        h3.h3_attention(d, r, st.q, st.k, st.v, st.o, qn_w=st.W["qn_w"], kn_w=st.W["kn_w"], pos=st.pos,
+                        flags=st.qk_flags)
+        mark(3, 1)
         mark(4, 0); h3.h3_gated_residual(d, r, st.x, st.o, st.W["Wo"], mod, h3.H3_MSA); mark(4, 1)
         mark(5, 0); h3.h3_adaln_norm_modulate(d, r, st.x, mod, h3.H3_MLP, st.xm); mark(5, 1)
         mark(6, 0); h3.h3_ffn_swiglu(d, r, st.x, st.xm, st.W["Wgu"], st.W["Wd"], mod, st.ws); mark(6, 1)
@@ -385,6 +391,7 @@ def run_ours(args, w):
                    "ffn": w.F, "text_tokens": w.n_text, "audio_tokens": w.audio_channels * w.n_audio,
                    "video_tokens": st.n_video, "video_latent": [w.T_lat, w.H_lat, w.W_lat, w.C_lat],
                    "parallelism": f"replicas x{world} (independent sequences)",
+                   "qk_norm_rope": "attention prologue" if st.qk_flags == 0 else "QKV epilogue",
                    "l2": "inputs larger than L2: %.0f MB of weights + %.0f MB residual stream read per step" % (
                        sum(t.numel() * 2 for t in W.values()) / 1e6, Lp * w.D * 4 / 1e6)},
         "roofline": {"bound": "tensor", "kernel": dominant,
@@ -710,7 +717,15 @@ def run_only(args, w):
     r = h3.h3_make_ranges(w.n_text, w.audio_channels * w.n_audio, w.T_lat * (w.H_lat // 2) * (w.W_lat // 2))
     Lp = r.L_pad
     mod = rnd(3, 6, w.D, std=0.1, dt=torch.float32)
-    if args.only in ("attention", "attention_raw"):
+    if args.only == "attention_prologue":
+        # raw N(0, 1) q, k (as the QKV call writes them without its norm and
+        # RoPE) with norm weights and seeded positions: the prologue kernel
+        q, k, v = (rnd(w.H, Lp, 128) for _ in range(3))
+        qn, kn = rnd(128, std=0.1) + 1, rnd(128, std=0.1) + 1
+        pos = torch.randint(0, 64, (Lp, 3), generator=g, device=dev).float()
+        o = torch.empty(Lp, w.I, dtype=torch.bfloat16, device=dev)
+        fn = lambda: h3.h3_attention(d, r, q, k, v, o, qn_w=qn, kn_w=kn, pos=pos, flags=0)
+    elif args.only in ("attention", "attention_raw"):
         # q, k rows as the QKV call leaves them: RMS-normalised and scaled by
         # the norm weights (attention then runs its split-softmax kernel);
         # attention_raw: unnormalised N(0, 1) rows, no norm weights (the
@@ -862,11 +877,15 @@ def main():
     ap.add_argument("--layers", type=int, default=50)
     ap.add_argument("--sp", action="store_true",
                     help="sequence parallelism: one sequence split over the job's ranks (a separate line)")
+    ap.add_argument("--qk-prologue", action="store_true",
+                    help="the per-head Q/K RMSNorm + RoPE in attention's prologue (raw q, k from the QKV call) "
+                         "instead of the QKV epilogue")
     ap.add_argument("--e4m3", action="store_true",
                     help="the block step with its four GEMMs in e4m3 (a separate line; one GPU)")
     ap.add_argument("--qk-e4m3", action="store_true",
                     help="with --e4m3: q and k cross to attention as e4m3 codes (Q K^T on e4m3 MMAs)")
-    ap.add_argument("--only", default=None, choices=["attention", "attention_raw", "qkv", "out", "ffn", "ln", "euler"],
+    ap.add_argument("--only", default=None, choices=["attention", "attention_raw", "attention_prologue", "qkv", "out",
+                                                     "ffn", "ln", "euler"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--heads", type=int, default=None, help="with --only: this many heads instead of the workload's")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

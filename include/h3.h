@@ -52,7 +52,9 @@ enum h3_status {
   H3_ERR_ALIGN = -3,       /* pointer not 16-byte aligned */
   H3_ERR_UNSUPPORTED = -4, /* head_dim != 128, D % 64 != 0, F % 128 != 0, ... */
   H3_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
-  H3_ERR_TIMEOUT = -6      /* a device-side wait gave up (see h3_device_status) */
+  H3_ERR_TIMEOUT = -6,     /* a device-side wait gave up (see h3_device_status) */
+  H3_ERR_BOUND = -7        /* attention with its norm and RoPE in the prologue met scores
+                              outside its static bound (see h3_attention, h3_device_status) */
 };
 
 enum h3_modality { H3_TEXT = 0, H3_AUDIO = 1, H3_VIDEO = 2 };
@@ -60,7 +62,12 @@ enum h3_branch { H3_MSA = 0, H3_MLP = 1 };
 
 /* h3_qkv_qknorm_mrope / h3_attention flag: Q/K RMSNorm and RoPE are applied
  * in the QKV GEMM epilogue (once per token), and h3_attention consumes the
- * already-rotated q, k.  Required in this version. */
+ * already-rotated q, k (the library's default placement, the faster one).
+ * Without it on both calls, the QKV call writes q, k raw and h3_attention
+ * applies the norm and RoPE in its prologue: each Q tile once per CTA and
+ * each K tile as it lands in shared memory ([shouss] §3.2 fixes the order,
+ * norm then RoPE, not the kernel that takes them).  The two placements give
+ * the same result up to the bf16 rounding of the raw q, k. */
 #define H3_QK_NORM_ROPE_IN_QKV 1
 /* With h3_qkv_qknorm_mrope_e4m3 / h3_attention / h3_block_forward_e4m3 only:
  * q and k are passed between the QKV call and attention as e4m3 codes (see
@@ -142,6 +149,8 @@ int h3_adaln_norm_modulate(const h3_dims* dims, const h3_ranges* ranges, const f
  * head_dim splits into t | h | w sections (rope_t, rope_h, rope_w); pair
  * (2i, 2i+1) of a section of width d turns by pos_axis * theta^(-2i/d)
  * ([shouss] §3.2: per-head RMSNorm then positional encoding; [gojay] §7.4).
+ * Without the flag q and k are written as the GEMM leaves them (rounded to
+ * bf16) and qn_w, kn_w, pos are not read (they may be NULL).
  *   pos [L_pad][3] fp32;  q, k, v out: head-major [H][L_pad][128] bf16. */
 int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* xm, const h3_bf16* Wqkv,
                         const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags, h3_bf16* q,
@@ -149,8 +158,16 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
 
 /* A6.  o = softmax(q k^T / sqrt(128)) v per head over all L valid tokens,
  * non-causal; keys >= L are masked ([shouss] §5).  q, k, v: head-major
- * [H][L_pad][128] bf16 as written by h3_qkv_qknorm_mrope (flags must carry
- * H3_QK_NORM_ROPE_IN_QKV; pos is unused and may be NULL).
+ * [H][L_pad][128] bf16 as written by h3_qkv_qknorm_mrope with the same
+ * H3_QK_NORM_ROPE_IN_QKV setting.
+ * Without H3_QK_NORM_ROPE_IN_QKV: q, k are raw; qn_w, kn_w and pos
+ * [L_pad][3] fp32 are required, and the split-softmax kernel normalises and
+ * rotates them in its prologue (four extra warps, one row each) before
+ * taking the same bounded softmax as below.  Nothing recomputes a CTA whose
+ * bound fails there: it leaves NaN in its first output element and
+ * h3_device_status then returns H3_ERR_BOUND (code 2).  The bound holds by
+ * construction for max|qn_w| * max|kn_w| <= 3.6.
+ * With the flag, pos is unused and may be NULL:
  *   qn_w, kn_w: the norm weights q and k were normalised with, or both NULL.
  *     Given (bf16 q, k), the softmax needs no running maximum: every score
  *     lies within sqrt(128) max|qn_w| max|kn_w| of 0, so the exponentials are

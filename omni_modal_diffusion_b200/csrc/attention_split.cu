@@ -56,16 +56,25 @@ using attn_detail::TILE;
 using attn_detail::TILE_BYTES;
 using attn_detail::TMEM_COLS;
 
-constexpr int NUM_THREADS = 18 * 32;
 constexpr int SVS = 2;  // V stages
-template <bool QK8>
+// PRO: q and k arrive raw (as the QKV GEMM leaves them) and the kernel takes
+// their per-head RMSNorm and 3-D RoPE in its prologue: four more warps
+// normalise and rotate each Q tile once and each K tile as it lands in
+// shared memory, before the MMA warp may read it.
+template <bool QK8, bool PRO = false>
 struct SLayout {
+  static_assert(!(QK8 && PRO), "the prologue takes bf16 q, k");
+  static constexpr int WARPS = PRO ? 22 : 18;
+  static constexpr int THREADS = WARPS * 32;
   static constexpr int QK_TILE = QK8 ? TILE_BYTES / 2 : TILE_BYTES;  // a Q or K tile (e4m3: 128-byte rows)
   static constexpr int SQ = 0;                                        // 2 query tiles
   static constexpr int SK = SQ + 2 * QK_TILE;                         // 2 stages
   static constexpr int SV = SK + 2 * QK_TILE;                         // SVS stages
   static constexpr int SBAR = SV + SVS * TILE_BYTES;
-  static constexpr int BYTES = SBAR + 256 + 1024;
+  // PRO: rotation frequency and axis of each of the 64 pairs, the two norm
+  // weights as fp32
+  static constexpr int SMISC = SBAR + 256;
+  static constexpr int BYTES = SMISC + (PRO ? 1536 : 0) + 1024;
   // [2 tiles][2 halves][128 rows] row sums (2 KB), written after a warp's key
   // loop: over the K stage that held K(nkv - 2), whose last S MMA completed
   // before any tile's last S (the other stage may still feed the other
@@ -93,12 +102,13 @@ __device__ __forceinline__ bf16* sentinel_ptr(const AttnOut& out, int grow, int 
   return out.shard[owner] + (long)(grow - owner * out.L_shard) * out.ld + (out.head0 + h) * 128;
 }
 
-template <bool QK8>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <bool QK8, bool PRO>
+__global__ void __launch_bounds__(SLayout<QK8, PRO>::THREADS, 1)
     attention_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnOut out, int H,
-                           int L, int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w) {
-  using Y = SLayout<QK8>;
+                           int L, int L_pad, float scale_log2, const bf16* qn_w, const bf16* kn_w,
+                           const __grid_constant__ attn_detail::AttnRope rope) {
+  using Y = SLayout<QK8, PRO>;
   constexpr int SQ = Y::SQ, SK = Y::SK, SV = Y::SV, SBAR = Y::SBAR, SSUM = Y::SSUM, QK_TILE = Y::QK_TILE;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -121,6 +131,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   float* bound = reinterpret_cast<float*>(bars + 21);
   int* cta_bad = reinterpret_cast<int*>(bars + 22);
   float* qk_scale = reinterpret_cast<float*>(bars + 23);  // QK8: dequantisation of S
+  uint64_t* q_ready = bars + 24;  // PRO: both Q tiles normalised and rotated (4 prologue warps)
+  uint64_t* k_ready = bars + 25;  // PRO: [2] the K stage normalised and rotated (4 prologue warps)
+  float* pro_freq = reinterpret_cast<float*>(smem + Y::SMISC);  // PRO: [64]
+  float* pro_qw = pro_freq + 64;                                 // PRO: [128] qn_w
+  float* pro_kw = pro_qw + 128;                                  // PRO: [128] kn_w
+  uint8_t* pro_axis = reinterpret_cast<uint8_t*>(pro_kw + 128);  // PRO: [64]
   float* lsum = reinterpret_cast<float*>(smem + SSUM + (((L + TILE - 1) / TILE) & 1) * QK_TILE);  // [t][hf][row]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -147,6 +163,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&v_empty[s], 1);
     }
     mbar_init(drain, 1);
+    if (PRO) {
+      mbar_init(q_ready, 4);
+      mbar_init(&k_ready[0], 4);
+      mbar_init(&k_ready[1], 4);
+    }
     mbar_init(&sums_done[0], 8 * nt);
     mbar_init(&sums_done[1], 8 * nt);
     *cta_bad = 0;
@@ -178,6 +199,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (QK8) *qk_scale = ((11.3137085f * mq) / 448.0f) * ((11.3137085f * mk) / 448.0f);
     }
   }
+  if (PRO && warp >= 18) {
+    // the norm weights as fp32, and each pair's rotation: pair i of the
+    // section of width d it falls in (t | h | w) turns by theta^(-2i/d) per
+    // unit of that axis' position (the QKV epilogue's table)
+    const int i = threadIdx.x - 18 * 32;  // 0 .. 127
+    pro_qw[i] = __bfloat162float(qn_w[i]);
+    pro_kw[i] = __bfloat162float(kn_w[i]);
+    if (i < 64) {
+      const int pt = rope.rope_t / 2, ph = rope.rope_h / 2;
+      int ax, i_sec, d_sec;
+      if (i < pt) { ax = 0; i_sec = i; d_sec = rope.rope_t; }
+      else if (i < pt + ph) { ax = 1; i_sec = i - pt; d_sec = rope.rope_h; }
+      else { ax = 2; i_sec = i - pt - ph; d_sec = rope.rope_w; }
+      pro_freq[i] = powf(rope.theta, -2.0f * (float)i_sec / (float)d_sec);
+      pro_axis[i] = (uint8_t)ax;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -188,7 +226,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (!fast) {
     // the bound is too wide for p to stay normal: leave the CTA to the
     // recomputing launch
-    if (threadIdx.x == 0) *sentinel_ptr(out, qt0 * TILE, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
+    if (threadIdx.x == 0) {
+      *sentinel_ptr(out, qt0 * TILE, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
+      if (PRO) atomicCAS(&g_h3_device_error, 0, 2);  // no launch recomputes it
+    }
   } else if (warp == 0) {
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, nt * QK_TILE);
@@ -248,7 +289,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         umma_bf16_tmem_a(tmem + t * 256 + 128, tmem + t * 256 + (kk >> 2) * 64 + (kk & 3) * 8,
                          vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j | kk) != 0 ? 1u : 0u);
     };
-    bool ok = mbar_wait_warp(q_full, 0) && mbar_wait_warp(&k_full[0], 0);
+    // PRO: Q and each K stage are read once the prologue warps have
+    // normalised and rotated them
+    uint64_t* q_in = PRO ? q_ready : q_full;
+    uint64_t* k_in = PRO ? k_ready : k_full;
+    bool ok = mbar_wait_warp(q_in, 0) && mbar_wait_warp(&k_in[0], 0);
     if (ok) {
       tc_fence_after();
       issue_s(0, 0);
@@ -261,7 +306,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // waiting for tile 0's P, so that each tile's P -> P V path holds one
       // wait (measured 3% faster than waiting for each just before its MMAs)
       ok = mbar_wait_warp(&v_full[j % SVS], (j / SVS) & 1) &&
-           (!more || mbar_wait_warp(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1));
+           (!more || mbar_wait_warp(&k_in[(j + 1) & 1], ((j + 1) >> 1) & 1));
       for (int t = 0; t < nt && ok; ++t) {
         if (!mbar_wait_warp(&p_full[t], j & 1)) { ok = false; break; }
         tc_fence_after();
@@ -276,6 +321,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       umma_commit(&v_empty[j % SVS]);
     }
     drain_mmas(drain);
+  } else if (PRO && warp >= 18) {
+    // One row per thread: RMSNorm (fp32, weights and eps of the QKV
+    // epilogue) then RoPE of row r of both Q tiles once, and of row r of
+    // every K tile as it lands; the row is read from and written back to its
+    // 128-byte-swizzled place (16-byte chunk c of row r at c ^ (r % 8)).
+    const int r = (warp - 18) * 32 + lane;
+    auto prep_row = [&](uint8_t* tile, int grow, const float* w) {
+      uint8_t* rowp = tile + r * 128;
+      const int sw = r & 7;
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4*>(rowp + (c >> 3) * HALF_BYTES + (((c & 7) ^ sw) << 4));
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b2[e]);
+          ss = fmaf(f.x, f.x, ss);
+          ss = fmaf(f.y, f.y, ss);
+        }
+      }
+      const float inv = rsqrtf(ss * (1.0f / 128.0f) + rope.eps);
+      float p3[3] = {0.f, 0.f, 0.f};
+      if (grow < L_pad) {
+        p3[0] = rope.pos[(long)grow * 3 + 0];
+        p3[1] = rope.pos[(long)grow * 3 + 1];
+        p3[2] = rope.pos[(long)grow * 3 + 2];
+      }
+#pragma unroll 2
+      for (int c = 0; c < 16; ++c) {
+        uint4* addr = reinterpret_cast<uint4*>(rowp + (c >> 3) * HALF_BYTES + (((c & 7) ^ sw) << 4));
+        uint4 u = *addr;
+        __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int d = c * 8 + e * 2;  // the pair (d, d + 1), pair index d / 2
+          const float2 f = __bfloat1622float2(b2[e]);
+          const float a = f.x * inv * w[d], bb = f.y * inv * w[d + 1];
+          const int ax = pro_axis[d >> 1];
+          const float pa = ax == 0 ? p3[0] : (ax == 1 ? p3[1] : p3[2]);
+          float sn, cs;
+          rope_sincos(pa * pro_freq[d >> 1], &sn, &cs);
+          b2[e] = __floats2bfloat162_rn(a * cs - bb * sn, a * sn + bb * cs);
+        }
+        *addr = u;
+      }
+    };
+    bool ok = mbar_wait_warp(q_full, 0);
+    if (ok) {
+      for (int t = 0; t < nt; ++t) prep_row(sQ + t * QK_TILE, (t == 0 ? qt0 : qt1) * TILE + r, pro_qw);
+      fence_proxy_async_smem();  // the MMAs read these rows through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait_warp(&k_full[st], (j >> 1) & 1)) break;
+      prep_row(sK + st * QK_TILE, j * TILE + r, pro_kw);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&k_ready[st]);
+    }
   } else if (((warp - 2) >> 3) < nt) {
     const int t = (warp - 2) >> 3;         // query tile
     const int hf = ((warp - 2) >> 2) & 1;  // key half of every key tile
@@ -364,7 +471,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const bool redo = *reinterpret_cast<volatile int*>(cta_bad) != 0;
       if (redo) {
-        if (t == 0 && hf == 0 && r == 0) *sentinel_ptr(out, grow, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
+        if (t == 0 && hf == 0 && r == 0) {
+          *sentinel_ptr(out, grow, h) = __ushort_as_bfloat16((unsigned short)0x7FC0);
+          if (PRO) atomicCAS(&g_h3_device_error, 0, 2);  // no launch recomputes it
+        }
       } else {
         const float inv = (grow < L) ? 1.0f / l : 0.0f;
         bf16* dst = sentinel_ptr(out, grow, h);
@@ -401,20 +511,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 cudaError_t launch_attention_split(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                    const attn_detail::AttnOut& out, dim3 grid, int H, int L, int L_pad,
                                    float scale_log2, const bf16* qn_w, const bf16* kn_w, bool qk8,
-                                   cudaStream_t stream) {
-  static unsigned long long attr_done[2] = {0, 0};
-  const void* kfn = qk8 ? reinterpret_cast<const void*>(attn_split::attention_split_kernel<true>)
-                        : reinterpret_cast<const void*>(attn_split::attention_split_kernel<false>);
-  cudaError_t e = ensure_smem_attr(kfn, qk8 ? attn_split::SLayout<true>::BYTES : attn_split::SLayout<false>::BYTES,
-                                   &attr_done[qk8 ? 1 : 0]);
+                                   const attn_detail::AttnRope* rope, cudaStream_t stream) {
+  using namespace attn_split;
+  static unsigned long long attr_done[3] = {0, 0, 0};
+  const attn_detail::AttnRope r = rope ? *rope : attn_detail::AttnRope{nullptr, 0, 0, 0, 0.f, 0.f};
+  const int which = rope ? 2 : (qk8 ? 1 : 0);
+  const void* kfn = which == 2 ? reinterpret_cast<const void*>(attention_split_kernel<false, true>)
+                    : which == 1 ? reinterpret_cast<const void*>(attention_split_kernel<true, false>)
+                                 : reinterpret_cast<const void*>(attention_split_kernel<false, false>);
+  const int bytes = which == 2 ? SLayout<false, true>::BYTES
+                    : which == 1 ? SLayout<true, false>::BYTES
+                                 : SLayout<false, false>::BYTES;
+  cudaError_t e = ensure_smem_attr(kfn, bytes, &attr_done[which]);
   if (e != cudaSuccess) return e;
-  if (qk8)
-    attn_split::attention_split_kernel<true><<<grid, attn_split::NUM_THREADS, attn_split::SLayout<true>::BYTES, stream>>>(
-        tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w);
+  if (which == 2)
+    attention_split_kernel<false, true><<<grid, SLayout<false, true>::THREADS, bytes, stream>>>(
+        tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w, r);
+  else if (which == 1)
+    attention_split_kernel<true, false><<<grid, SLayout<true, false>::THREADS, bytes, stream>>>(
+        tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w, r);
   else
-    attn_split::attention_split_kernel<false>
-        <<<grid, attn_split::NUM_THREADS, attn_split::SLayout<false>::BYTES, stream>>>(tq, tk, tv, out, H, L, L_pad,
-                                                                                       scale_log2, qn_w, kn_w);
+    attention_split_kernel<false, false><<<grid, SLayout<false, false>::THREADS, bytes, stream>>>(
+        tq, tk, tv, out, H, L, L_pad, scale_log2, qn_w, kn_w, r);
   return cudaGetLastError();
 }
 

@@ -105,6 +105,14 @@ struct AttnOut {
   bf16* shard[8];
 };
 
+// RMSNorm + 3-D RoPE taken in the attention prologue (split kernel, PRO):
+// positions [L_pad][3], the t | h | w section widths, the base, the norm eps
+struct AttnRope {
+  const float* pos;
+  int rope_t, rope_h, rope_w;
+  float theta, eps;
+};
+
 // QK8: Q and K are e4m3 codes of q * 448 / (sqrt(128) max|qn_w|) and of
 // k * 448 / (sqrt(128) max|kn_w|); S = Q K^T is taken with kind::f8f6f4 MMAs
 // and the two scales folded into the softmax scale.  P V stays bf16.
@@ -504,7 +512,7 @@ bool make_tmap_e4m3(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 cudaError_t launch_attention_split(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                    const attn_detail::AttnOut& out, dim3 grid, int H, int L, int L_pad,
                                    float scale_log2, const bf16* qn_w, const bf16* kn_w, bool qk8,
-                                   cudaStream_t stream);
+                                   const attn_detail::AttnRope* rope, cudaStream_t stream);
 
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
   const bool qk8 = p.qk8 != 0;
@@ -543,12 +551,22 @@ cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream) {
 #ifndef H3_ATTN_SPLIT
 #define H3_ATTN_SPLIT 1
 #endif
+  if (p.prologue) {
+    // raw q, k: the split kernel normalises and rotates them in its
+    // prologue.  No recomputing launch follows (the general kernel takes q, k
+    // as given): a CTA whose static bound fails leaves its sentinel and code
+    // 2 in the device error word.
+    if (qk8 || p.qn_w == nullptr || p.kn_w == nullptr || p.pos == nullptr) return cudaErrorInvalidValue;
+    attn_detail::AttnRope rope{p.pos, p.rope_t, p.rope_h, p.rope_w, p.theta, p.eps_qk};
+    return launch_attention_split(tq, tk, tv, out, grid, p.H, p.L, p.L_pad, p.scale_log2, p.qn_w, p.kn_w, false,
+                                  &rope, stream);
+  }
   if (H3_ATTN_SPLIT && p.qn_w != nullptr && p.kn_w != nullptr) {
     // the split-softmax kernel on normalised q, k (bf16 or e4m3 codes); then
     // this kernel on the CTAs it left (usually none: each such CTA returns
     // at once)
     aerr = launch_attention_split(tq, tk, tv, out, grid, p.H, p.L, p.L_pad, p.scale_log2, p.qn_w, p.kn_w, qk8,
-                                  stream);
+                                  nullptr, stream);
     if (aerr != cudaSuccess) return aerr;
     if (qk8)
       attention_tc_kernel<true><<<grid, attn_detail::NUM_THREADS, Layout<true>::BYTES, stream>>>(

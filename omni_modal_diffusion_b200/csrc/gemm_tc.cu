@@ -246,7 +246,7 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
                                         const uint8_t* axis_of_pair, const float* qk_inv, int h_lo = 0,
                                         int h_hi = 2) {
   float p3[3] = {0.f, 0.f, 0.f};
-  if (m < e.L_pad) {
+  if (m < e.L_pad && !e.qk_raw) {  // raw q, k: pos is not read (it may be null)
     p3[0] = e.pos[(long)m * 3 + 0];
     p3[1] = e.pos[(long)m * 3 + 1];
     p3[2] = e.pos[(long)m * 3 + 2];
@@ -260,7 +260,8 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
     const uint32_t th = tb + half * 128;
     float inv = 1.0f;
     const bf16* w = part == 0 ? e.qn_w : e.kn_w;
-    if (part < 2) {
+    const bool norm_rope = part < 2 && !e.qk_raw;
+    if (norm_rope) {
       float ss = 0.f;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -290,7 +291,7 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
       ld_chunk(th + c * 32, v);
       tmem_wait_ld();
       scale_chunk(e, v, m, n + c * 32);
-      if (part < 2) {
+      if (norm_rope) {
 #pragma unroll
         for (int d = 0; d < 32; d += 8) {
           const uint4 wv = __ldg(reinterpret_cast<const uint4*>(w + c * 32 + d));

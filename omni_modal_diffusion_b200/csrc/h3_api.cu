@@ -288,19 +288,21 @@ int h3_qkv_qknorm_mrope(const h3_dims* dims, const h3_ranges* ranges, const h3_b
   H3_TRACE();
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
-  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
-    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
   if (flags & ~H3_QK_NORM_ROPE_IN_QKV)
     return fail(H3_ERR_UNSUPPORTED, "%s: e4m3 q/k output needs h3_qkv_qknorm_mrope_e4m3", __func__);
+  const bool in_qkv = (flags & H3_QK_NORM_ROPE_IN_QKV) != 0;
   H3_REQUIRE_PTR(xm);
   H3_REQUIRE_PTR(Wqkv);
-  H3_REQUIRE_PTR(qn_w);
-  H3_REQUIRE_PTR(kn_w);
-  H3_REQUIRE_PTR(pos);
+  if (in_qkv) {  // without the flag q, k leave raw and qn_w, kn_w, pos go to h3_attention instead
+    H3_REQUIRE_PTR(qn_w);
+    H3_REQUIRE_PTR(kn_w);
+    H3_REQUIRE_PTR(pos);
+  }
   H3_REQUIRE_PTR(q);
   H3_REQUIRE_PTR(k);
   H3_REQUIRE_PTR(v);
   GemmProblem p = qkv_problem(dims, ranges, xm, Wqkv, qn_w, kn_w, pos, q, k, v);
+  p.epi.qk_raw = in_qkv ? 0 : 1;
   cudaError_t e = launch_gemm(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "h3_qkv_qknorm_mrope");
   return ok();
@@ -310,19 +312,29 @@ int h3_attention(const h3_dims* dims, const h3_ranges* ranges, const h3_bf16* q,
                  const h3_bf16* v, const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
                  h3_bf16* o, void* stream) {
   H3_TRACE();
-  (void)pos;
   H3_CHECK(check_dims(dims, __func__));
   H3_CHECK(check_ranges(ranges, __func__));
-  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
-    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
   if (flags & ~(H3_QK_NORM_ROPE_IN_QKV | H3_QK_E4M3)) return fail(H3_ERR_UNSUPPORTED, "%s: unknown flags", __func__);
+  if ((flags & H3_QK_E4M3) && !(flags & H3_QK_NORM_ROPE_IN_QKV))
+    return fail(H3_ERR_UNSUPPORTED, "%s: e4m3 q, k are written by the QKV epilogue after its norm and RoPE", __func__);
   H3_REQUIRE_PTR(q);
   H3_REQUIRE_PTR(k);
   H3_REQUIRE_PTR(v);
   H3_REQUIRE_PTR(o);
   AttnProblem p;
   memset(&p, 0, sizeof(p));
-  if (flags & H3_QK_E4M3) {  // q, k: e4m3 codes whose scales follow from qn_w, kn_w
+  if (!(flags & H3_QK_NORM_ROPE_IN_QKV)) {  // raw q, k: RMSNorm and RoPE in attention's prologue
+    H3_REQUIRE_PTR(qn_w);
+    H3_REQUIRE_PTR(kn_w);
+    H3_REQUIRE_PTR(pos);
+    p.prologue = 1;
+    p.pos = pos;
+    p.rope_t = dims->rope_t;
+    p.rope_h = dims->rope_h;
+    p.rope_w = dims->rope_w;
+    p.theta = dims->theta;
+    p.eps_qk = dims->eps_qk;
+  } else if (flags & H3_QK_E4M3) {  // q, k: e4m3 codes whose scales follow from qn_w, kn_w
     H3_REQUIRE_PTR(qn_w);
     H3_REQUIRE_PTR(kn_w);
     p.qk8 = 1;
@@ -621,6 +633,9 @@ int h3_device_status(void* stream, int* code_out) {
     if (e != cudaSuccess) return cuda_fail(e, "h3_device_status: clear");
   }
   if (code_out) *code_out = code;
+  if (code == 2)
+    return fail(H3_ERR_BOUND, "h3_device_status: attention with its norm and RoPE in the prologue met scores "
+                              "outside the bound its norm weights give (those rows hold NaN)");
   if (code != 0) return fail(H3_ERR_TIMEOUT, "h3_device_status: a device-side wait gave up (code %d)", code);
   return ok();
 }

@@ -43,6 +43,9 @@ struct GemmEpilogue {
   // to [H][L_pad][128] bytes) of value * 448 / (sqrt(128) max|w|), w the
   // head's norm weight; v stays bf16
   int qk_e4m3;
+  // EPI_QKV with qk_raw: q and k are written as they leave the GEMM (no
+  // RMSNorm, no RoPE), for attention to take both in its prologue
+  int qk_raw;
   // EPI_UNPATCH: token grid (T, Ht, Wt), latent channels
   int Ht, Wt, C_lat;
   // EPI_STORE_F32 / EPI_UNPATCH with euler != 0: out holds a latent that
@@ -108,6 +111,14 @@ struct AttnProblem {
   int qk8;
   const bf16* qn_w;
   const bf16* kn_w;
+  // prologue != 0: q, k are raw (the QKV GEMM without its norm and RoPE),
+  // and attention applies the per-head RMSNorm (weights qn_w, kn_w, eps) and
+  // the 3-D RoPE (positions pos [L_pad][3], sections rope_t | rope_h |
+  // rope_w, base theta) in its prologue
+  int prologue;
+  const float* pos;
+  int rope_t, rope_h, rope_w;
+  float theta, eps_qk;
 };
 cudaError_t launch_attention(const AttnProblem& p, cudaStream_t stream);
 

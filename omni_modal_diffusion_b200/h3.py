@@ -16,6 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libh3.so")
 
 H3_OK, H3_ERR_NULL, H3_ERR_SHAPE, H3_ERR_ALIGN, H3_ERR_UNSUPPORTED, H3_ERR_CUDA, H3_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+H3_ERR_BOUND = -7
 H3_TEXT, H3_AUDIO, H3_VIDEO = 0, 1, 2
 H3_MSA, H3_MLP = 0, 1
 H3_QK_NORM_ROPE_IN_QKV = 1
@@ -314,7 +315,7 @@ def h3_euler_step_bf16(lat, vel, sigma: float, sigma_next: float, lat_bf16, stre
 def h3_device_status(stream=None) -> int:
     code = ctypes.c_int(0)
     rc = lib().h3_device_status(_stream(stream), ctypes.byref(code))
-    if rc not in (H3_OK, H3_ERR_TIMEOUT):
+    if rc not in (H3_OK, H3_ERR_TIMEOUT, H3_ERR_BOUND):
         _check(rc)
     return code.value
 

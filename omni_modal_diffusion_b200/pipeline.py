@@ -27,6 +27,9 @@ class H3BlockStep:
         self.w = w
         self.device = torch.device(device)
         self.dims = h3.make_dims(w.D, w.H, w.F, head_dim=w.head_dim, rope=w.rope_split)
+        # where the per-head Q/K RMSNorm + RoPE run: the QKV epilogue (the
+        # default, once per token) or, with 0, attention's prologue
+        self.qk_flags = h3.H3_QK_NORM_ROPE_IN_QKV
         self.n_video = w.T_lat * (w.H_lat // 2) * (w.W_lat // 2)
         self.n_audio_tok = w.audio_channels * w.n_audio
         self.ranges = h3.h3_make_ranges(w.n_text, self.n_audio_tok, self.n_video)
@@ -71,8 +74,9 @@ class H3BlockStep:
         d, r = self.dims, self.ranges
         h3.h3_adaln_norm_modulate(d, r, self.x, mod, h3.H3_MSA, self.xm, stream=stream)
         h3.h3_qkv_qknorm_mrope(d, r, self.xm, W["Wqkv"], W["qn_w"], W["kn_w"], self.pos, self.q, self.k, self.v,
-                               stream=stream)
-        h3.h3_attention(d, r, self.q, self.k, self.v, self.o, qn_w=W["qn_w"], kn_w=W["kn_w"], stream=stream)
+                               flags=self.qk_flags, stream=stream)
+        h3.h3_attention(d, r, self.q, self.k, self.v, self.o, qn_w=W["qn_w"], kn_w=W["kn_w"], pos=self.pos,
+                        flags=self.qk_flags, stream=stream)
         h3.h3_gated_residual(d, r, self.x, self.o, W["Wo"], mod, h3.H3_MSA, stream=stream)
         h3.h3_adaln_norm_modulate(d, r, self.x, mod, h3.H3_MLP, self.xm, stream=stream)
         h3.h3_ffn_swiglu(d, r, self.x, self.xm, W["Wgu"], W["Wd"], mod, self.ws, stream=stream)

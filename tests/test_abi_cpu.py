@@ -87,9 +87,15 @@ def test_validation_rejects_bad_arguments_without_launch(lib):
     assert lib.h3_euler_step(None, None, -1, 0.0, 0.0, None) == h3.H3_ERR_SHAPE
     assert lib.h3_euler_step(None, None, 0, 0.0, 0.0, None) == h3.H3_OK
     assert lib.h3_euler_step(ctypes.c_void_p(16), None, 4, 0.0, 0.0, None) == h3.H3_ERR_NULL
-    # the QKV / attention calls need the norm+RoPE placement flag
+    # without the norm+RoPE placement flag attention takes them in its
+    # prologue and needs the norm weights and the positions; e4m3 q, k need
+    # the flag (the QKV epilogue writes the codes after its norm and RoPE)
     z = ctypes.c_void_p(16)
     assert lib.h3_attention(ctypes.byref(d), ctypes.byref(r), z, z, z, None, None, None, 0, z, None) == \
+        h3.H3_ERR_NULL
+    assert lib.h3_attention(ctypes.byref(d), ctypes.byref(r), z, z, z, z, z, None, 0, z, None) == h3.H3_ERR_NULL
+    assert b"pos" in lib.h3_last_error()
+    assert lib.h3_attention(ctypes.byref(d), ctypes.byref(r), z, z, z, z, z, z, h3.H3_QK_E4M3, z, None) == \
         h3.H3_ERR_UNSUPPORTED
     # e4m3 q, k: attention needs the norm weights (their scales), unknown
     # flags are refused, and the bf16 QKV call cannot write e4m3 codes
