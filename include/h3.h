@@ -306,7 +306,9 @@ typedef struct h3_block_buffers {
  * (MLP), h3_ffn_swiglu, in the order of [shouss] §3 (norm + modality
  * shift/scale -> shared attention + gate + residual -> norm + shift/scale ->
  * shared gated FFN + gate + residual).  Same arguments and errors as those
- * calls; nothing is launched if any argument is invalid. */
+ * calls; nothing is launched if any argument is invalid.  flags: 0 or
+ * H3_QK_NORM_ROPE_IN_QKV, passed to the QKV and attention calls (where the
+ * Q/K norm and RoPE run). */
 int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, const float* mod, const float* pos,
                      const h3_block_weights* w, const h3_block_buffers* buf, int flags, void* stream);
 

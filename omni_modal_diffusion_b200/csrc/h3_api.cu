@@ -584,8 +584,7 @@ int h3_block_forward(const h3_dims* dims, const h3_ranges* ranges, float* x, con
   H3_CHECK(check_ranges(ranges, __func__));
   if (!w) return fail(H3_ERR_NULL, "%s: weights is NULL", __func__);
   if (!buf) return fail(H3_ERR_NULL, "%s: buffers is NULL", __func__);
-  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
-    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  if (flags & ~H3_QK_NORM_ROPE_IN_QKV) return fail(H3_ERR_UNSUPPORTED, "%s: unknown flags", __func__);
   H3_REQUIRE_PTR(x);
   H3_REQUIRE_PTR(mod);
   H3_REQUIRE_PTR(pos);

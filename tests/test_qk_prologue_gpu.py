@@ -199,3 +199,33 @@ def test_full_length_prologue_sampled_rows():
     ref = O.attention_rows(qn, kn, vo)
     check_close(got, ref, "prologue attention L=124016 rows")
     assert float(o[L:].float().abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("w", WORKLOADS, ids=lambda w: w.name)
+def test_block_with_prologue_placement(w):
+    """The whole block with the norm and RoPE in attention's prologue
+    (h3_block_forward and the pipeline with flags 0) against the oracle's
+    block: the block bound on the output, the branch-delta bound of the
+    default placement on its delta."""
+    inp = S.make_inputs(w)
+    st = H3BlockStep(w, device=DEV, weights=inp)
+    st.qk_flags = 0
+    st.embed(*(to_dev_bf16(inp[kk], DEV) for kk in ("text", "video", "audio")))
+    mod = torch.from_numpy(inp["mod"]).to(DEV)
+    r, pos = oracle_ranges_and_pos(w)
+    L = r["L"]
+    x0_dev = st.x.clone()
+    st.block(mod)
+    assert h3.h3_device_status() == 0
+    x_pipe = to_np(st.x)[:L]
+    # the same block through the C-ABI block call with flags 0
+    st.x.copy_(x0_dev)
+    h3.h3_block_forward(st.dims, st.ranges, st.x, mod, st.pos, h3.block_weights(st.W),
+                        h3.block_buffers(st.xm, st.q, st.k, st.v, st.o, st.ws), flags=0)
+    assert h3.h3_device_status() == 0
+    assert np.array_equal(to_np(st.x)[:L], x_pipe)
+    x0 = O.embed(inp["text"], inp["video"], inp["audio"], inp["W_text"], inp["W_vid"], inp["W_aud"], r)
+    ref = O.block_forward(x0, inp["mod"], r, pos, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"], inp["Wgu"],
+                          inp["Wd"], w.H)
+    check_close(x_pipe, ref, "block output, prologue placement")
+    check_close(x_pipe - x0, ref - x0, "block delta, prologue placement", max_rel_rms=5e-2)
