@@ -131,15 +131,6 @@ __device__ __forceinline__ bool mbar_wait_spin_warp(uint64_t* bar, uint32_t pari
   return __all_sync(0xffffffffu, mbar_wait_spin(bar, parity));
 }
 
-// Warp-uniform form with a vote-first fast path: every lane probes the phase
-// once and the warp votes; only a warp that finds it incomplete enters the
-// bounded wait loop.  No lane leaves before the others (both votes take the
-// whole warp), and an already completed phase costs one probe and one vote.
-__device__ __forceinline__ bool mbar_wait_warp_fast(uint64_t* bar, uint32_t parity) {
-  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
-}
-
 // ------------------------------------------------------------ clusters (CTA pairs)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
