@@ -487,7 +487,8 @@ int h3_sp_make_layout(const h3_dims* dims, const h3_ranges* global, int n_ranks,
 /* Device pointers of every rank's exchange buffers (index = rank):
  *   q[g], k[g], v[g]: rank g's [H/N][L_total][128] bf16 (head-major; global
  *                     row order, so the attention of rank g sees the whole
- *                     sequence for its heads)
+ *                     sequence for its heads); with H3_QK_E4M3, q[g] and
+ *                     k[g] hold one-byte e4m3 codes in the same layout
  *   o[g]:             rank g's [L_shard][H * 128] bf16 attention output */
 typedef struct h3_sp_peers {
   h3_bf16* q[H3_SP_MAX_RANKS];
@@ -503,13 +504,25 @@ int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3
                            const h3_bf16* xm, const h3_bf16* Wqkv, const h3_bf16* qn_w, const h3_bf16* kn_w,
                            const float* pos, int flags, const h3_sp_peers* peers, void* stream);
 
+/* NEXT-1 with NEXT-2: h3_qkv_qknorm_mrope_sp on e4m3 operands (xq [L_shard][D]
+ * codes with per-row scales xs, Wq [3I][D] codes with per-output-channel
+ * scales Ws, as h3_qkv_qknorm_mrope_e4m3).  With flags & H3_QK_E4M3 the q, k
+ * that cross to the head-group ranks are e4m3 codes (half the bytes of
+ * bf16; scales from qn_w, kn_w), and every rank's h3_attention_sp then takes
+ * the same flag. */
+int h3_qkv_qknorm_mrope_sp_e4m3(const h3_dims* dims, const h3_ranges* shard, const h3_sp_layout* layout,
+                                const h3_e4m3* xq, const float* xs, const h3_e4m3* Wq, const float* Ws,
+                                const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
+                                const h3_sp_peers* peers, void* stream);
+
 /* A6 for this rank's H/N heads over all L tokens (its q, k, v =
  * peers->q/k/v[rank], filled by every rank's h3_qkv_qknorm_mrope_sp), with
  * output row R (global) written to peers->o[R / L_shard], row R % L_shard,
  * columns of head (rank H/N + h): attention and the second all-to-all in
  * one kernel.  Rows >= L are written as 0.  qn_w, kn_w: as for
  * h3_attention (the norm weights q and k were normalised with, selecting
- * the split-softmax kernel, or both NULL). */
+ * the split-softmax kernel, or both NULL; required with H3_QK_E4M3, where q
+ * and k are e4m3 codes). */
 int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers,
                     const h3_bf16* qn_w, const h3_bf16* kn_w, int flags, void* stream);
 

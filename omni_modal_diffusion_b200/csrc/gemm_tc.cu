@@ -319,7 +319,14 @@ __device__ __forceinline__ void epi_qkv(const GemmEpilogue& e, uint32_t tb, int 
 #pragma unroll
         for (int d = 0; d < 32; d += 4)
           w4[d / 4] = cvt_e4m3x2(v[d] * inv, v[d + 1] * inv) | (cvt_e4m3x2(v[d + 2] * inv, v[d + 3] * inv) << 16);
-        uint8_t* dst8 = reinterpret_cast<uint8_t*>(part == 0 ? e.q : e.k) + ((long)h * e.L_pad + m) * 128 + c * 32;
+        uint8_t* dst8;
+        if (e.sp_n > 0) {  // sequence parallel: the codes go straight to the head group's rank
+          const int g = h / e.sp_heads, hl = h - g * e.sp_heads;
+          dst8 = reinterpret_cast<uint8_t*>(part == 0 ? e.sp_q[g] : e.sp_k[g]) +
+                 ((long)hl * e.sp_L_total + e.sp_row0 + m) * 128 + c * 32;
+        } else {
+          dst8 = reinterpret_cast<uint8_t*>(part == 0 ? e.q : e.k) + ((long)h * e.L_pad + m) * 128 + c * 32;
+        }
         reinterpret_cast<uint4*>(dst8)[0] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         reinterpret_cast<uint4*>(dst8)[1] = make_uint4(w4[4], w4[5], w4[6], w4[7]);
       } else if (dst) {

@@ -1,6 +1,6 @@
 // Sequence parallelism (Ulysses) for the block: the layout of a rank's shard
 // and the two exchange points, each fused into the kernel that produces the
-// data.  "MiniMax-H3 paper reading" (gojay.top) §7.2 gives Ulysses degree 4
+// data (bf16 q, k, v, or with e4m3 operands e4m3 q, k codes and bf16 v).  "MiniMax-H3 paper reading" (gojay.top) §7.2 gives Ulysses degree 4
 // as the trunk's deployment; the all-to-all structure (tokens -> heads before
 // attention, heads -> tokens after it) is the method's, the fusion is ours:
 //   - h3_qkv_qknorm_mrope_sp: the QKV epilogue stores head group g of the
@@ -118,6 +118,44 @@ int h3_qkv_qknorm_mrope_sp(const h3_dims* dims, const h3_ranges* shard, const h3
   return ok();
 }
 
+int h3_qkv_qknorm_mrope_sp_e4m3(const h3_dims* dims, const h3_ranges* shard, const h3_sp_layout* layout,
+                                const h3_e4m3* xq, const float* xs, const h3_e4m3* Wq, const float* Ws,
+                                const h3_bf16* qn_w, const h3_bf16* kn_w, const float* pos, int flags,
+                                const h3_sp_peers* peers, void* stream) {
+  H3_TRACE();
+  H3_CHECK(check_dims(dims, __func__));
+  H3_CHECK(check_ranges(shard, __func__));
+  H3_CHECK(check_layout(dims, layout, __func__));
+  if (shard->L_pad != layout->L_shard)
+    return fail(H3_ERR_SHAPE, "%s: shard L_pad (%d) != layout L_shard (%d)", __func__, shard->L_pad, layout->L_shard);
+  if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
+    return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
+  if (flags & ~(H3_QK_NORM_ROPE_IN_QKV | H3_QK_E4M3)) return fail(H3_ERR_UNSUPPORTED, "%s: unknown flags", __func__);
+  H3_REQUIRE_PTR(xq);
+  H3_REQUIRE_PTR(xs);
+  H3_REQUIRE_PTR(Wq);
+  H3_REQUIRE_PTR(Ws);
+  H3_REQUIRE_PTR(qn_w);
+  H3_REQUIRE_PTR(kn_w);
+  H3_REQUIRE_PTR(pos);
+  H3_CHECK(check_peers(peers, layout->n_ranks, true, false, __func__));
+  GemmProblem p = with_e4m3(qkv_problem(dims, shard, xq, Wq, qn_w, kn_w, pos, nullptr, nullptr, nullptr), xs, Ws);
+  GemmEpilogue& e = p.epi;
+  e.qk_e4m3 = (flags & H3_QK_E4M3) ? 1 : 0;
+  e.sp_n = layout->n_ranks;
+  e.sp_heads = layout->heads;
+  e.sp_L_total = layout->L_total;
+  e.sp_row0 = layout->row0;
+  for (int g = 0; g < layout->n_ranks; ++g) {
+    e.sp_q[g] = reinterpret_cast<bf16*>(peers->q[g]);
+    e.sp_k[g] = reinterpret_cast<bf16*>(peers->k[g]);
+    e.sp_v[g] = reinterpret_cast<bf16*>(peers->v[g]);
+  }
+  cudaError_t err = launch_gemm(p, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "h3_qkv_qknorm_mrope_sp_e4m3");
+  return ok();
+}
+
 int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp_peers* peers,
                     const h3_bf16* qn_w, const h3_bf16* kn_w, int flags, void* stream) {
   H3_TRACE();
@@ -125,20 +163,20 @@ int h3_attention_sp(const h3_dims* dims, const h3_sp_layout* layout, const h3_sp
   H3_CHECK(check_layout(dims, layout, __func__));
   if (!(flags & H3_QK_NORM_ROPE_IN_QKV))
     return fail(H3_ERR_UNSUPPORTED, "%s: flags must include H3_QK_NORM_ROPE_IN_QKV in this version", __func__);
-  if (flags & ~H3_QK_NORM_ROPE_IN_QKV)
-    return fail(H3_ERR_UNSUPPORTED, "%s: only H3_QK_NORM_ROPE_IN_QKV (e4m3 q/k are not sequence parallel)", __func__);
+  if (flags & ~(H3_QK_NORM_ROPE_IN_QKV | H3_QK_E4M3)) return fail(H3_ERR_UNSUPPORTED, "%s: unknown flags", __func__);
   H3_CHECK(check_peers(peers, layout->n_ranks, false, true, __func__));
   const int r = layout->rank;
   if (!peers->q[r] || !peers->k[r] || !peers->v[r])
     return fail(H3_ERR_NULL, "%s: this rank's q, k, v buffers are required", __func__);
   if (!aligned16(peers->q[r]) || !aligned16(peers->k[r]) || !aligned16(peers->v[r]))
     return fail(H3_ERR_ALIGN, "%s: this rank's q, k, v buffers must be 16-byte aligned", __func__);
-  if (qn_w || kn_w) {
+  if (qn_w || kn_w || (flags & H3_QK_E4M3)) {  // e4m3 codes: their scales follow from the norm weights
     H3_REQUIRE_PTR(qn_w);
     H3_REQUIRE_PTR(kn_w);
   }
   AttnProblem p;
   memset(&p, 0, sizeof(p));
+  p.qk8 = (flags & H3_QK_E4M3) ? 1 : 0;
   p.qn_w = reinterpret_cast<const bf16*>(qn_w);
   p.kn_w = reinterpret_cast<const bf16*>(kn_w);
   p.q = reinterpret_cast<const bf16*>(peers->q[r]);

@@ -32,7 +32,8 @@ EXPORTS = (
     "h3_euler_step_bf16", "h3_selftest_wait_timeout",
     "h3_quantize_rows_e4m3", "h3_adaln_norm_modulate_e4m3", "h3_qkv_qknorm_mrope_e4m3", "h3_gated_residual_e4m3",
     "h3_ffn_e4m3_workspace_bytes", "h3_ffn_swiglu_e4m3", "h3_block_forward_e4m3",
-    "h3_sp_make_layout", "h3_qkv_qknorm_mrope_sp", "h3_attention_sp", "h3_text_refine",
+    "h3_sp_make_layout", "h3_qkv_qknorm_mrope_sp", "h3_qkv_qknorm_mrope_sp_e4m3", "h3_attention_sp",
+    "h3_text_refine",
 )
 H3_SP_MAX_RANKS = 8
 H3_FFN_STATIC_WS_BYTES = 32 * 1024 * 1024
@@ -133,6 +134,8 @@ def lib() -> ctypes.CDLL:
             "h3_sp_make_layout": (ci, [pd, pr, ci, ci, ctypes.POINTER(SPLayout), pr]),
             "h3_qkv_qknorm_mrope_sp": (ci, [pd, pr, ctypes.POINTER(SPLayout), vp, vp, vp, vp, vp, ci,
                                             ctypes.POINTER(SPPeers), vp]),
+            "h3_qkv_qknorm_mrope_sp_e4m3": (ci, [pd, pr, ctypes.POINTER(SPLayout), vp, vp, vp, vp, vp, vp, vp, ci,
+                                                 ctypes.POINTER(SPPeers), vp]),
             "h3_attention_sp": (ci, [pd, ctypes.POINTER(SPLayout), ctypes.POINTER(SPPeers), vp, vp, ci, vp]),
             "h3_text_refine": (ci, [pd, pr, vp, ci, ctypes.POINTER(ctypes.c_void_p), vp,
                                     ctypes.POINTER(BlockWeights), ctypes.POINTER(BlockBuffers), ci, vp]),
@@ -407,9 +410,10 @@ def h3_sp_make_layout(dims, global_ranges, n_ranks: int, rank: int):
     return lay, shard
 
 
-def sp_peers(q=None, k=None, v=None, o=None) -> SPPeers:
+def sp_peers(q=None, k=None, v=None, o=None, qk_e4m3: bool = False) -> SPPeers:
     """Peer table from per-rank lists of CUDA tensors (index = rank); a list
-    may be None when the call does not use it."""
+    may be None when the call does not use it.  qk_e4m3: q and k are uint8
+    tensors of e4m3 codes."""
     p = SPPeers()
     for name, ts in (("q", q), ("k", k), ("v", v), ("o", o)):
         if ts is None:
@@ -417,8 +421,9 @@ def sp_peers(q=None, k=None, v=None, o=None) -> SPPeers:
         if len(ts) > H3_SP_MAX_RANKS:
             raise ValueError(f"at most {H3_SP_MAX_RANKS} ranks")
         arr = getattr(p, name)
+        dt = U8 if qk_e4m3 and name in ("q", "k") else BF16
         for i, t in enumerate(ts):
-            arr[i] = _ptr(t, BF16, f"{name}[{i}]").value
+            arr[i] = _ptr(t, dt, f"{name}[{i}]").value
     return p
 
 
@@ -428,6 +433,14 @@ def h3_qkv_qknorm_mrope_sp(dims, shard, layout, xm, Wqkv, qn_w, kn_w, pos, peers
                                         _ptr(xm, BF16, "xm"), _ptr(Wqkv, BF16, "Wqkv"), _ptr(qn_w, BF16, "qn_w"),
                                         _ptr(kn_w, BF16, "kn_w"), _ptr(pos, F32, "pos"), flags, ctypes.byref(peers),
                                         _stream(stream)))
+
+
+def h3_qkv_qknorm_mrope_sp_e4m3(dims, shard, layout, xq, xs, Wq, Ws, qn_w, kn_w, pos, peers: SPPeers,
+                                flags=H3_QK_NORM_ROPE_IN_QKV, stream=None):
+    _check(lib().h3_qkv_qknorm_mrope_sp_e4m3(ctypes.byref(dims), ctypes.byref(shard), ctypes.byref(layout),
+                                             _ptr(xq, U8, "xq"), _ptr(xs, F32, "xs"), _ptr(Wq, U8, "Wq"),
+                                             _ptr(Ws, F32, "Ws"), _ptr(qn_w, BF16, "qn_w"), _ptr(kn_w, BF16, "kn_w"),
+                                             _ptr(pos, F32, "pos"), flags, ctypes.byref(peers), _stream(stream)))
 
 
 def h3_attention_sp(dims, layout, peers: SPPeers, qn_w=None, kn_w=None, flags=H3_QK_NORM_ROPE_IN_QKV,

@@ -55,13 +55,15 @@ class SPProcessRank:
     (shard of the residual stream, exchange buffers) with a peer table over
     every rank's buffers, opened through CUDA IPC."""
 
-    def __init__(self, w, dims, global_ranges, device, group=None):
+    def __init__(self, w, dims, global_ranges, device, group=None, e4m3: bool = False, qk_e4m3: bool = False):
         self.world = dist.get_world_size(group)
         self.index = dist.get_rank(group)
         self.group = group
         self.rank = sp.SPRank(w, dims, global_ranges, self.world, self.index, device)
         r = self.rank
-        self._peers = sp.exchange_peer_tensors({"q": r.q, "k": r.k, "v": r.v, "o": r.o}, group)
+        if e4m3:  # e4m3 block buffers; with qk_e4m3 the q, k exchange buffers hold codes
+            r.alloc_e4m3(qk_e4m3)
+        self._peers = sp.exchange_peer_tensors({"q": r.exchange_q(), "k": r.exchange_k(), "v": r.v, "o": r.o}, group)
         r.set_peers(self._peers["q"], self._peers["k"], self._peers["v"], self._peers["o"])
         self.barrier = ProcessBarrier(device, group)
 
@@ -77,6 +79,10 @@ class SPProcessRank:
         """One block on this rank's shard; every rank calls it with the same
         block (its own shard of the residual stream in `self.rank.x`)."""
         sp.block_forward([self.rank], mod, W, barrier=self.barrier, stream=stream)
+
+    def block_forward_e4m3(self, mod, W8, stream=None):
+        """One block with e4m3 GEMMs (constructed with e4m3=True)."""
+        sp.block_forward_e4m3([self.rank], mod, W8, barrier=self.barrier, stream=stream)
 
     def close(self):
         """Release the peers' buffers before anyone frees its own."""

@@ -137,3 +137,49 @@ def test_sp_argument_errors():
     empty = h3.SPPeers()
     with pytest.raises(h3.H3Error):
         h3.h3_attention_sp(d, lay, empty)
+
+
+@pytest.mark.parametrize("qk_e4m3", [False, True], ids=["qk_bf16", "qk_e4m3"])
+@pytest.mark.parametrize("w,n_ranks", [(RAGGED, 2), (LONG, 4)], ids=["ragged2", "long4"])
+def test_sp_e4m3_block_matches_single_gpu_e4m3_block(w, n_ranks, qk_e4m3):
+    """Sequence parallelism with the block's GEMMs on e4m3 operands, and with
+    qk_e4m3 the q, k crossing to the head-group ranks as e4m3 codes: the
+    sharded block equals the single-sequence e4m3 block bit for bit (the
+    same codes, scales and accumulation order per row)."""
+    inp = S.make_inputs(w)
+    st = H3BlockStep(w, weights=inp)
+    text, video, audio = (to_dev_bf16(inp[k], st.device) for k in ("text", "video", "audio"))
+    mod = torch.from_numpy(inp["mod"]).to(st.device)
+    st.embed(text, video, audio)
+    W8 = st.quantize_block_weights_e4m3()
+    st.alloc_e4m3()
+    x0 = st.x.clone()
+    pos = st.pos.clone()
+    L = st.ranges.L
+
+    ranks = [sp.SPRank(w, st.dims, st.ranges, n_ranks, r, DEV) for r in range(n_ranks)]
+    for r in ranks:
+        r.alloc_e4m3(qk_e4m3)
+        r.x.zero_()
+        r.pos.zero_()
+        lo, hi = r.rows.start, min(r.rows.stop, st.ranges.L_pad)
+        if hi > lo:
+            r.x[: hi - lo].copy_(x0[lo:hi])
+            r.pos[: hi - lo].copy_(pos[lo:hi])
+        for t in (r.v, r.o):
+            t.fill_(float("nan"))
+        if qk_e4m3:
+            r.q8.fill_(0x7F)  # e4m3 NaN codes: a row the exchange misses shows
+            r.k8.fill_(0x7F)
+        else:
+            r.q.fill_(float("nan"))
+            r.k.fill_(float("nan"))
+    sp.link_local(ranks)
+    sp.block_forward_e4m3(ranks, mod, W8)
+    st.block_e4m3(mod, W8, qk_e4m3=qk_e4m3)
+    torch.cuda.synchronize()
+    assert h3.h3_device_status() == 0
+    x_sp = torch.cat([r.x for r in ranks], 0)[:L]
+    assert torch.equal(x_sp, st.x[:L]), "sharded e4m3 block differs from the single-sequence e4m3 block"
+    for r in ranks:
+        assert torch.all(r.x[r.shard.L:] == 0)
