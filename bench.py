@@ -659,7 +659,11 @@ def run_sp(args, w):
              randn(w.audio_channels, w.n_audio, w.C_audio))
     mod = randn(3, 6, w.D, std=0.1, dtype=torch.float32)
     L = st.ranges.L
-    me = SPProcessRank(w, st.dims, st.ranges, dev)
+    e4m3 = bool(getattr(args, "e4m3", False))
+    qk8 = e4m3 and bool(getattr(args, "qk_e4m3", False))
+    W8 = st.quantize_block_weights_e4m3() if e4m3 else None
+    me = SPProcessRank(w, st.dims, st.ranges, dev, e4m3=e4m3, qk_e4m3=qk8)
+    fwd = (lambda: me.block_forward_e4m3(mod, W8)) if e4m3 else (lambda: me.block_forward(mod, W))
     r = me.rank
     r.x.zero_()
     r.pos.zero_()
@@ -672,12 +676,12 @@ def run_sp(args, w):
     me.barrier()
     for _ in range(args.warmup):
         r.x.copy_(x0)
-        me.block_forward(mod, W)
+        fwd()
     me.barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        me.block_forward(mod, W)
+        fwd()
     t1.record(stream)
     me.barrier()
     ms = t0.elapsed_time(t1) / args.steps
@@ -693,11 +697,15 @@ def run_sp(args, w):
     return {"metric": "packed tokens/s per Omni block, sequence-parallel (Ulysses) over the job's GPUs",
             "value": round(L / (ms / 1e3), 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/text, N(0,0.02) weights)",
+            "vs_baseline": None,
+            "dtype": ("e4m3 GEMMs" + (", e4m3 Q K^T" if qk8 else "") + ", bf16 P V") if e4m3 else "bf16",
+            "data": "synthetic (seeded N(0,1) latents/text, N(0,0.02) weights)",
             "config": {"workload": w.name, "packed_tokens": L, "parallelism": f"ulysses sp{world}",
-                       "L_shard": me.layout.L_shard, "heads_per_rank": me.layout.heads},
+                       "L_shard": me.layout.L_shard, "heads_per_rank": me.layout.heads,
+                       "q_k_exchange": "e4m3 codes" if qk8 else "bf16"},
             "tflops": round(fl / (ms / 1e3) / 1e12, 1),
-            "gpu_launches": 8 * args.steps,   # LN, QKV, attention (split + fixup), out-projection, LN, FFN x2
+            # LN, QKV, attention (split + fixup), out-projection, LN, FFN x2 (e4m3: + 2 row quantisers)
+            "gpu_launches": (10 if e4m3 else 8) * args.steps,
             "barriers_per_block": 2}
 
 
