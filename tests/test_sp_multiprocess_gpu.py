@@ -28,7 +28,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, out_dir, n_blocks):
+def _rank_main(rank, world, port, out_dir, n_blocks, e4m3=False):
     import datetime
 
     import torch.distributed as dist
@@ -46,7 +46,10 @@ def _rank_main(rank, world, port, out_dir, n_blocks):
     st = H3BlockStep(w, device=dev, weights=inp)
     st.embed(*(to_dev_bf16(inp[k], dev) for k in ("text", "video", "audio")))
     mod = torch.from_numpy(inp["mod"]).to(dev)
-    me = SPProcessRank(w, st.dims, st.ranges, dev)
+    W8 = st.quantize_block_weights_e4m3() if e4m3 else None
+    if e4m3:
+        st.alloc_e4m3()
+    me = SPProcessRank(w, st.dims, st.ranges, dev, e4m3=e4m3, qk_e4m3=e4m3)
     r = me.rank
     r.x.zero_()
     r.pos.zero_()
@@ -55,15 +58,24 @@ def _rank_main(rank, world, port, out_dir, n_blocks):
     r.pos[: hi - lo].copy_(st.pos[lo:hi])
     for t in (r.q, r.k, r.v, r.o):
         t.fill_(float("nan"))
+    if e4m3:
+        r.q8.fill_(0x7F)              # e4m3 NaN codes: a row the exchange misses shows
+        r.k8.fill_(0x7F)
     me.barrier()                      # every rank's buffers initialised before any peer store
     for _ in range(n_blocks):
-        me.block_forward(mod, st.W)
+        if e4m3:
+            me.block_forward_e4m3(mod, W8)
+        else:
+            me.block_forward(mod, st.W)
     torch.cuda.synchronize()
     status = h3.h3_device_status()
     np.save(os.path.join(out_dir, f"x_rank{rank}.npy"), r.x.cpu().numpy())
     if rank == 0:
         for _ in range(n_blocks):
-            st.block(mod)
+            if e4m3:
+                st.block_e4m3(mod, W8, qk_e4m3=True)
+            else:
+                st.block(mod)
         torch.cuda.synchronize()
         np.save(os.path.join(out_dir, "x_single.npy"), st.x.cpu().numpy())
     me.close()
@@ -94,3 +106,20 @@ def test_sp_two_processes_one_gpu(tmp_path, n_blocks):
         x = O.block_forward(x, inp["mod"], r_o, pos_o, inp["Wqkv"], inp["qn_w"], inp["kn_w"], inp["Wo"], inp["Wgu"],
                             inp["Wd"], w.H)
     check_close(x_sp, x, f"two-process sequence-parallel block output ({n_blocks} block(s))")
+
+
+@pytest.mark.timeout(600)
+def test_sp_two_processes_one_gpu_e4m3(tmp_path):
+    """The same with e4m3 GEMMs and e4m3 q, k codes over the exchange: the
+    two processes' shards equal the single-sequence e4m3 block bit for bit."""
+    import torch.multiprocessing as mp
+
+    from omni_modal_diffusion_b200 import build
+    build.build()
+    world = 2
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path), 1, True), nprocs=world, join=True)
+    L = oracle_ranges_and_pos(RAGGED)[0]["L"]
+    shards = [np.load(tmp_path / f"x_rank{g}.npy") for g in range(world)]
+    x_sp = np.concatenate(shards, 0)[:L]
+    x_single = np.load(tmp_path / "x_single.npy")[:L]
+    assert np.array_equal(x_sp, x_single), "two-process sharded e4m3 block differs from the single-sequence one"
