@@ -103,6 +103,12 @@ TRAFFIC = {
     # them); q, k, v, o alone are 7.11 GB, the rest is K and V re-read by
     # CTAs that started at different times
     ("768x1792_15s", "attention_split_kernel"): 15.49e9,
+    # mean over the block's four pair-GEMM launches at 32,160 tokens
+    # (39.65 GB / 4: A panels re-read per pass of the concurrent tiles, B once
+    # per band, the outputs); every term grows with the rows, so 124,016
+    # tokens take that times 124,016 / 32,160
+    ("768x1344_5s", "gemm_tc_kernel"): 9.91e9,
+    ("768x1792_15s", "gemm_tc_kernel"): 38.2e9,
 }
 
 
