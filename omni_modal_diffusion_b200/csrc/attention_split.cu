@@ -15,6 +15,8 @@
 //   Warp 1       TMEM owner and MMA issuer
 //   Warps 2-17   softmax: tile t = (w - 2) / 8, key half hf = ((w - 2) / 4) % 2,
 //                lane quarter w % 4 (the quarter a warp may access in TMEM)
+//   Warps 18-21  PRO only: RMSNorm + RoPE of the raw Q tiles and of each K
+//                tile in shared memory, one row per thread
 //
 // The MMA warp holds one wait on each tile's path from P to P V: the tile's
 // eight softmax warps arrive on one barrier, and the waits for V(j) and
@@ -44,6 +46,12 @@
 // exponent scale.  Rounding q and k to e4m3 (3 mantissa bits) moves each
 // element by at most 2^-4 of itself, so the bound takes the factor
 // (1 + 2^-4)^2 = 1.129: B = 16.32 * 1.14 max|qn_w| max|kn_w|.
+//
+// PRO: the alternative placement of the per-head Q/K RMSNorm + RoPE, in this
+// kernel's prologue instead of the QKV epilogue (raw q, k in).  It redoes
+// the normalisation and rotation of every key row for every CTA of its head
+// and measures 2.4-2.7x slower per call; the library's default placement is
+// the QKV epilogue.
 #include "h3_internal.cuh"
 #include "ptx.cuh"
 
