@@ -103,6 +103,8 @@ TRAFFIC = {
     # them); q, k, v, o alone are 7.11 GB, the rest is K and V re-read by
     # CTAs that started at different times
     ("768x1792_15s", "attention_split_kernel"): 15.49e9,
+    # the same with e4m3 q, k codes: 201.6 MB + 47.9 MB for 2 heads, times 28
+    ("768x1792_15s", "attention_split_kernel<e4m3 QK>"): 6.99e9,
     # mean over the block's four pair-GEMM launches at 32,160 tokens
     # (39.65 GB / 4: A panels re-read per pass of the concurrent tiles, B once
     # per band, the outputs); every term grows with the rows, so 124,016
@@ -739,6 +741,21 @@ def run_only(args, w):
         pos = torch.randint(0, 64, (Lp, 3), generator=g, device=dev).float()
         o = torch.empty(Lp, w.I, dtype=torch.bfloat16, device=dev)
         fn = lambda: h3.h3_attention(d, r, q, k, v, o, qn_w=qn, kn_w=kn, pos=pos, flags=0)
+    elif args.only == "attention_qk8":
+        # q, k as the e4m3 QKV epilogue leaves them: codes of the normalised
+        # rows times 448 / (sqrt(128) max|w|) (input generation: torch's
+        # float8 conversion), v bf16
+        qn, kn = rnd(128, std=0.1) + 1, rnd(128, std=0.1) + 1
+        def codes(wt):
+            xf = rnd(w.H, Lp, 128).float()
+            xf = xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + 1e-6) * wt.float()
+            inv = 448.0 / (128 ** 0.5 * float(wt.float().abs().max()))
+            return (xf * inv).to(torch.float8_e4m3fn).view(torch.uint8)
+        q8, k8 = codes(qn), codes(kn)
+        v = rnd(w.H, Lp, 128)
+        o = torch.empty(Lp, w.I, dtype=torch.bfloat16, device=dev)
+        fl = h3.H3_QK_NORM_ROPE_IN_QKV | h3.H3_QK_E4M3
+        fn = lambda: h3.h3_attention(d, r, q8, k8, v, o, qn_w=qn, kn_w=kn, flags=fl)
     elif args.only in ("attention", "attention_raw"):
         # q, k rows as the QKV call leaves them: RMS-normalised and scaled by
         # the norm weights (attention then runs its split-softmax kernel);
@@ -898,8 +915,8 @@ def main():
                     help="the block step with its four GEMMs in e4m3 (a separate line; one GPU)")
     ap.add_argument("--qk-e4m3", action="store_true",
                     help="with --e4m3: q and k cross to attention as e4m3 codes (Q K^T on e4m3 MMAs)")
-    ap.add_argument("--only", default=None, choices=["attention", "attention_raw", "attention_prologue", "qkv", "out",
-                                                     "ffn", "ln", "euler"],
+    ap.add_argument("--only", default=None, choices=["attention", "attention_raw", "attention_prologue",
+                                                     "attention_qk8", "qkv", "out", "ffn", "ln", "euler"],
                     help="launch only this call (small ncu captures); prints timing, no JSON contract line")
     ap.add_argument("--heads", type=int, default=None, help="with --only: this many heads instead of the workload's")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

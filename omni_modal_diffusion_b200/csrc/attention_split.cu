@@ -69,6 +69,16 @@ constexpr int SVS = 2;  // V stages
 // their per-head RMSNorm and 3-D RoPE in its prologue: four more warps
 // normalise and rotate each Q tile once and each K tile as it lands in
 // shared memory, before the MMA warp may read it.
+// e4m3 Q K^T: 2 of every 16 exponentials on the FMA pipe.  Measured per call
+// (TFLOP/s at 7,904 tokens / 124,016 tokens with 8 heads): 1,399 / 1,387 all
+// on MUFU; 1,504 / 1,446 with 2; 1,503 / 1,427 with 4; 1,495 / 1,418 with 6.
+// The bf16 kernel measured slower with any share (its tensor pipe, not
+// MUFU, is the busier unit), so it takes none.
+#ifndef H3_ATTN_SPLIT_QK8_POLY
+#define H3_ATTN_SPLIT_QK8_POLY 2
+#endif
+static_assert(H3_ATTN_SPLIT_QK8_POLY >= 0 && H3_ATTN_SPLIT_QK8_POLY <= 16 && H3_ATTN_SPLIT_QK8_POLY % 2 == 0,
+              "H3_ATTN_SPLIT_QK8_POLY: an even count of 0..16");
 template <bool QK8, bool PRO = false>
 struct SLayout {
   static_assert(!(QK8 && PRO), "the prologue takes bf16 q, k");
@@ -410,13 +420,28 @@ __global__ void __launch_bounds__(SLayout<QK8, PRO>::THREADS, 1)
     bool ok = true;
     // p = 2^(s scale_log2 - B) for 32 scores; their bf16 pairs into pk[16];
     // returns their sum (masked keys, -inf, give 0)
-    auto exp32 = [&](const float* s, uint32_t* pk) {
+    // QK8 with H3_ATTN_SPLIT_QK8_POLY: that many of every 16 exponentials on
+    // the FMA pipe (exp2_fma2), where the e4m3 S leaves the tensor pipe slack
+    // and the MUFU unit is the busier one; never on the last key tile (its
+    // masked keys must give exactly 0)
+    constexpr int kPoly = QK8 ? H3_ATTN_SPLIT_QK8_POLY : 0;
+    const float pa = sl2 * (1.0f / 252.0f), pb = (125.0f - B) * (1.0f / 252.0f);
+    (void)pa;
+    (void)pb;
+    auto exp32 = [&](const float* s, uint32_t* pk, auto poly_tag) {
+      constexpr int kP = decltype(poly_tag)::value;
       uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 32; c += 2) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nb2), x0, x1);
-        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        float p0, p1;
+        if (kP > 0 && (c & 15) < kP) {
+          f2_unpack(exp2_fma2(s[c], s[c + 1], pa, pb), p0, p1);
+        } else {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sc2, nb2), x0, x1);
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
         acc[(c >> 1) & 1] = f2_add(acc[(c >> 1) & 1], f2_pack(p0, p1));
         pk[c / 2] = pack_bf16x2(p0, p1);
       }
@@ -425,6 +450,8 @@ __global__ void __launch_bounds__(SLayout<QK8, PRO>::THREADS, 1)
       f2_unpack(acc[1], a2, a3);
       return (a0 + a1) + (a2 + a3);
     };
+    using NoPoly = std::integral_constant<int, 0>;
+    using Poly = std::integral_constant<int, kPoly>;
     for (int j = 0; j < nkv; ++j) {
       ok = mbar_wait_warp(&s_full[t], j & 1);
       if (!ok) break;
@@ -439,7 +466,11 @@ __global__ void __launch_bounds__(SLayout<QK8, PRO>::THREADS, 1)
         for (int c = 0; c < 32; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      float hs = exp32(s, pkA);
+      float hs;
+      if constexpr (kPoly == 0)
+        hs = exp32(s, pkA, NoPoly{});
+      else
+        hs = valid < 64 ? exp32(s, pkA, NoPoly{}) : exp32(s, pkA, Poly{});
       // P of keys [0, 32) of the half over its own first 16 score columns
       tmem_st16(tH, pkA);
       tmem_ld32(tH + 32, reinterpret_cast<uint32_t*>(s));
@@ -449,7 +480,10 @@ __global__ void __launch_bounds__(SLayout<QK8, PRO>::THREADS, 1)
         for (int c = 0; c < 32; ++c)
           if (c + 32 >= valid) s[c] = -INFINITY;
       }
-      hs += exp32(s, pkB);
+      if constexpr (kPoly == 0)
+        hs += exp32(s, pkB, NoPoly{});
+      else
+        hs += valid < 64 ? exp32(s, pkB, NoPoly{}) : exp32(s, pkB, Poly{});
       // P of keys [32, 64) of the half over score columns [16, 32), already read
       tmem_st16(tH + 16, pkB);
       tmem_wait_st();
