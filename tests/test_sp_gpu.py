@@ -140,7 +140,7 @@ def test_sp_argument_errors():
 
 
 @pytest.mark.parametrize("qk_e4m3", [False, True], ids=["qk_bf16", "qk_e4m3"])
-@pytest.mark.parametrize("w,n_ranks", [(RAGGED, 2), (LONG, 4)], ids=["ragged2", "long4"])
+@pytest.mark.parametrize("w,n_ranks", [(RAGGED, 2), (RAGGED, 3), (LONG, 4)], ids=["ragged2", "ragged3", "long4"])
 def test_sp_e4m3_block_matches_single_gpu_e4m3_block(w, n_ranks, qk_e4m3):
     """Sequence parallelism with the block's GEMMs on e4m3 operands, and with
     qk_e4m3 the q, k crossing to the head-group ranks as e4m3 codes: the
