@@ -103,8 +103,9 @@ TRAFFIC = {
     # them); q, k, v, o alone are 7.11 GB, the rest is K and V re-read by
     # CTAs that started at different times
     ("768x1792_15s", "attention_split_kernel"): 15.49e9,
-    # the same with e4m3 q, k codes: 201.6 MB + 47.9 MB for 2 heads, times 28
-    ("768x1792_15s", "attention_split_kernel<e4m3 QK>"): 6.99e9,
+    # the same with e4m3 q, k codes (2 of 16 exponentials on the FMA pipe):
+    # 178.3 MB + 48.0 MB for 2 heads, times 28
+    ("768x1792_15s", "attention_split_kernel<e4m3 QK>"): 6.34e9,
     # mean over the block's four pair-GEMM launches at 32,160 tokens
     # (39.65 GB / 4: A panels re-read per pass of the concurrent tiles, B once
     # per band, the outputs); every term grows with the rows, so 124,016
